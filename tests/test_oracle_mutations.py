@@ -1,0 +1,47 @@
+"""The oracle's pins catch planted mistakes.
+
+Each case copies oracle.c, plants one plausible mistake in the copy (a dropped
+scale, a flipped sign, a transposed operand, an off-by-one mask, a dropped term),
+builds it with gcc into a temporary library and runs the pin tests against it
+in a child process.  The pins must fail for every mutant.  Nothing here touches
+the real oracle build.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTANTS = {
+    "dk_scale_dropped": ("dk[(size_t)j * d + x] = c->scale * acc;", "dk[(size_t)j * d + x] = acc;"),
+    "ds_sign_flipped": ("(dP[(size_t)i * N + j] - D[i])", "(D[i] - dP[(size_t)i * N + j])"),
+    "causal_off_by_one": ("if ((flags & ORACLE_CAUSAL) && j > i) return 0;",
+                          "if ((flags & ORACLE_CAUSAL) && j >= i) return 0;"),
+    "dv_operand_transposed": ("acc += P[(size_t)i * N + j] * dout[(size_t)i * d + x];",
+                              "acc += P[(size_t)j * N + i] * dout[(size_t)i * d + x];"),
+    "lse_max_dropped": ("double lse = m + log(l);", "double lse = log(l);"),
+    "mask_index_transposed": ("!mask[(size_t)(i / blk) * nbk + (j / blk)]",
+                              "!mask[(size_t)(j / blk) * nbk + (i / blk)]"),
+    "scale_dropped_in_scores": ("srow[j] = scale * acc;", "srow[j] = acc;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found for {name}"
+    mut = src.replace(old, new)
+    cfile = tmp_path / "oracle_mut.c"
+    cfile.write_text(mut)
+    lib = tmp_path / "liboracle_mut.so"
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-I", os.path.join(ROOT, "oracle"),
+                    "-o", str(lib), str(cfile), "-lm", "-lpthread"], check=True)
+    env = dict(os.environ, ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
