@@ -1,0 +1,170 @@
+"""flash_fwd_b200 -- exact softmax attention on B200 (sm_100a).
+
+A thin ctypes binding over ``libfa_b200.so`` (declared in ``include/fa.h``).
+The functions below only marshal arguments: every step of the attention runs
+in the library's CUDA kernels.  PyTorch supplies device memory and streams.
+
+If the library has not been built the binding raises; there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FaError", "load_library", "library_path", "fa_fwd", "fa_fwd_blocksparse", "fa_bwd",
+    "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status",
+    "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK",
+]
+
+FA_BLOCK = 128
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+FA_F16, FA_BF16 = 0, 1
+_DTYPE = {torch.float16: FA_F16, torch.bfloat16: FA_BF16}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: status {status} ({fa_status_string(status)})")
+
+
+def library_path():
+    return os.path.join(_PKG, "libfa_b200.so")
+
+
+def load_library():
+    """Loads libfa_b200.so once; raises if it is missing."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m flash_fwd_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_bytes.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, i, vp]
+    lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_device_status.argtypes = []
+    lib.fa_version.argtypes = []
+    for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse,
+               lib.fa_last_device_status, lib.fa_version):
+        fn.restype = ctypes.c_int
+    _LIB = lib
+    return lib
+
+
+def fa_status_string(status):
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def fa_last_device_status():
+    return load_library().fa_last_device_status()
+
+
+def fa_version():
+    return load_library().fa_version()
+
+
+def fa_bwd_workspace_bytes(B, H, N, d):
+    return load_library().fa_bwd_workspace_bytes(B, H, N, d)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def _dtype(q):
+    if q.dtype not in _DTYPE:
+        raise ValueError("q, k, v must be float16 or bfloat16")
+    return _DTYPE[q.dtype]
+
+
+def _scale(scale, d):
+    return float(scale) if scale is not None else 1.0 / float(d) ** 0.5
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise FaError(rc, what)
+
+
+def fa_fwd(q, k, v, o, lse, causal=False, scale=None, stream=None):
+    """O and LSE of exact attention; all tensors [B, H, N, d] (lse [B, H, N] fp32)."""
+    B, H, N, d = _shape(q)
+    rc = load_library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                               _scale(scale, d), int(bool(causal)), _dtype(q), _stream(stream))
+    _check(rc, "fa_fwd")
+
+
+def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, causal=False, scale=None, stream=None):
+    B, H, N, d = _shape(q)
+    rc = load_library().fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask),
+                                           B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q),
+                                           _stream(stream))
+    _check(rc, "fa_fwd_blocksparse")
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, stream=None):
+    B, H, N, d = _shape(q)
+    rc = load_library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q), _stream(stream))
+    _check(rc, "fa_bwd")
+
+
+def fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask, causal=False, scale=None,
+                       stream=None):
+    B, H, N, d = _shape(q)
+    rc = load_library().fa_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _ptr(block_mask),
+                                           B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q),
+                                           _stream(stream))
+    _check(rc, "fa_bwd_blocksparse")
+
+
+def attention_fwd(q, k, v, causal=False, scale=None, block_mask=None, stream=None):
+    """Allocates O and LSE with torch and runs the forward; returns (o, lse)."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if block_mask is None:
+        fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    else:
+        fa_fwd_blocksparse(q, k, v, o, lse, block_mask, causal, scale, stream)
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, dout, lse, causal=False, scale=None, block_mask=None, workspace=None,
+                  stream=None):
+    """Allocates dQ, dK, dV (and the workspace unless given) and runs the backward."""
+    B, H, N, d = _shape(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    if block_mask is None:
+        fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal, scale, stream)
+    else:
+        fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask, causal, scale, stream)
+    return dq, dk, dv

@@ -1,0 +1,174 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA
+// descriptor encoding and kernel launches.  No device memory is allocated here.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// [BH][N][d] 16-bit tensor seen as a 3-D TMA map {d, N, BH} with 64 x rows x 1
+// boxes and 128-byte swizzle; rows past N read as zeros.
+int make_map(CUtensorMap *map, const void *base, int d, int N, long long BH, int dtype, int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return FA_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int check_common(int B, int H, int N, int d, float scale, int dtype) {
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    // grid.y holds query-block pairs (<= 65535)
+    if ((static_cast<long long>(N) + 255) / 256 > 65535) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+template <int D, int NQ, int NS, bool BF16>
+int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const fa::FwdParams &p,
+               int BH, cudaStream_t stream) {
+    using C = fa::FwdCfg<D, NQ, NS>;
+    auto kern = fa::fwd_kernel<D, NQ, NS, BF16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    dim3 grid(BH, (p.nqb + NQ - 1) / NQ);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool BF16>
+int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                 const fa::FwdParams &p, int BH, cudaStream_t s) {
+    switch (d) {
+        case 64: return launch_fwd<64, 2, 4, BF16>(mq, mk, mv, p, BH, s);
+        case 128: return launch_fwd<128, 2, 2, BF16>(mq, mk, mv, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, BF16>(mq, mk, mv, p, BH, s);
+        default: return FA_ERR_UNSUPPORTED;
+    }
+}
+
+int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, const uint8_t *mask, int B,
+             int H, int N, int d, float scale, int causal, int dtype, void *stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    const int BH = B * H;
+    CUtensorMap mq, mk, mv;
+    if ((rc = make_map(&mq, q, d, N, BH, dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, k, d, N, BH, dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, d, N, BH, dtype, 128)) != FA_OK) return rc;
+    fa::FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.mask = mask;
+    p.N = N;
+    p.nqb = (N + 127) / 128;
+    p.nkb = p.nqb;
+    p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
+    p.scale_log2 = scale * kLog2e;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dtype == FA_BF16 ? dispatch_fwd<true>(d, mq, mk, mv, p, BH, s)
+                            : dispatch_fwd<false>(d, mq, mk, mv, p, BH, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+                  float scale, int causal, int dtype, void *stream) {
+    return fwd_impl(q, k, v, o, lse, nullptr, B, H, N, d, scale, causal, dtype, stream);
+}
+
+FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const uint8_t *block_mask, int B, int H, int N, int d, float scale, int causal,
+                              int dtype, void *stream) {
+    if (!block_mask) return FA_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, o, lse, block_mask, B, H, N, d, scale, causal, dtype, stream);
+}
+
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128 && d != 256)) return 0;
+    return fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d);
+}
+
+FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+                  void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int N,
+                  int d, float scale, int causal, int dtype, void *stream) {
+    return fa::bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d,
+                         scale, causal, dtype, stream);
+}
+
+FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                              const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                              size_t workspace_bytes, const uint8_t *block_mask, int B, int H, int N, int d,
+                              float scale, int causal, int dtype, void *stream) {
+    if (!block_mask) return FA_ERR_INVALID_ARG;
+    return fa::bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, block_mask, B, H, N,
+                         d, scale, causal, dtype, stream);
+}
+
+FA_API const char *fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG: return "invalid argument";
+        case FA_ERR_UNSUPPORTED: return "unsupported shape";
+        case FA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case FA_ERR_WORKSPACE: return "workspace missing or too small";
+        case FA_ERR_CUDA: return "CUDA error";
+        case FA_ERR_TIMEOUT: return "kernel wait timed out";
+        default: return "unknown status";
+    }
+}
+
+FA_API int fa_last_device_status(void) {
+    int v = 0, zero = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, fa::g_dev_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(fa::g_dev_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return v;
+}
+
+FA_API int fa_version(void) { return 100; }
+
+}  // extern "C"

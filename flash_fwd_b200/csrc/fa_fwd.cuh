@@ -1,0 +1,453 @@
+// fa_fwd.cuh -- forward kernel of exact attention for sm_100a.
+//
+// What it computes: for every (batch, head) and query row i,
+//   O_i = sum_j softmax_j(scale * q_i . k_j) v_j,  LSE_i = ln sum_j exp(scale * q_i . k_j)
+// over the keys visible to i, with the online softmax of "FlashAttention
+// 深度解析" section 二: a running max m and sum l are corrected by
+// 2^(m_old - m_new) whenever a key tile raises the max, O stays unnormalised
+// and is divided by l once at the end (深度解析 section 四, deferred
+// normalisation).  S and P live only in tensor memory ("FlashAttention原理概览"
+// section 3.1: the intermediate S_ij and P_ij never reach device memory).
+//
+// Decomposition (the outer-Q / inner-K/V order of 深度解析 section 四): one
+// CTA owns NQ query tiles of 128 rows of one (batch, head) and streams the
+// kept 128-key tiles of K and V through an NS-stage shared-memory ring.
+//
+// Warp roles (a B200 design; the pages' own schedules target A100/H100):
+//   warps 0 .. 4*NQ-1   softmax: warpgroup t owns query tile t, one thread per
+//                       row.  It reads S_t from TMEM, masks, updates m and l,
+//                       rescales O_t in TMEM when m grew by more than 2^8
+//                       (exactness is kept because O and l share the stale m),
+//                       writes P_t (16-bit) back over S_t and signals the MMA warp.
+//   warp 4*NQ           TMA producer: Q tiles once, then K_j and V_j per stage.
+//   warp 4*NQ+1         MMA issuer (one elected lane): S_t = Q_t K_j^T (SS form)
+//                       and O_t += P_t V_j (P read from TMEM, TS form).  It owns
+//                       the 512-column TMEM allocation.
+// TMEM columns: S_t at [128 t, 128 t + 128) (P_t reuses its first 64 columns),
+// O_t at [256 + D t, 256 + D t + D).
+//
+// Scale handling: exp is evaluated as 2^(s * scale * log2 e - m), with the
+// running max m kept in that base-2 domain; LSE converts back to natural log.
+#pragma once
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+enum MaskMode : int { kDense = 0, kCausal = 1, kSparse = 2 };
+
+struct FwdParams {
+    void *o;                  // [BH][N][D] 16-bit
+    float *lse;               // [BH][N]
+    const uint8_t *mask;      // [nqb][nkb] block mask (kSparse)
+    int N;
+    int nqb;                  // query blocks of 128 rows
+    int nkb;                  // key blocks of 128 keys
+    int mode;                 // kCausal | kSparse bits
+    float scale_log2;         // scale * log2(e)
+};
+
+// Is key block j visible at all from query block rb?
+__device__ __forceinline__ bool block_kept(const FwdParams &p, int rb, int j) {
+    if (rb >= p.nqb || j >= p.nkb) return false;
+    if ((p.mode & kCausal) && j > rb) return false;
+    if ((p.mode & kSparse) && p.mask[static_cast<size_t>(rb) * p.nkb + j] == 0) return false;
+    return true;
+}
+
+// Walks, in increasing order, the key blocks kept by at least one of the CTA's
+// NQ query blocks (rb0, rb0 + 1).  Warp-collective: all 32 lanes call next().
+template <int NQ>
+struct KvIter {
+    int base = -32;
+    uint32_t b0 = 0, b1 = 0;
+    __device__ __forceinline__ bool next(const FwdParams &p, int rb0, int &j, uint32_t &flags) {
+        while ((b0 | b1) == 0u) {
+            base += 32;
+            if (base >= p.nkb) return false;
+            const int jj = base + static_cast<int>(lane_id());
+            b0 = __ballot_sync(0xffffffffu, block_kept(p, rb0, jj));
+            b1 = (NQ > 1) ? __ballot_sync(0xffffffffu, block_kept(p, rb0 + 1, jj)) : 0u;
+        }
+        const uint32_t u = b0 | b1;
+        const int b = __ffs(u) - 1;
+        flags = ((b0 >> b) & 1u) | (((b1 >> b) & 1u) << 1);
+        b0 &= ~(1u << b);
+        b1 &= ~(1u << b);
+        j = base + b;
+        return true;
+    }
+};
+
+template <int D, int NQ, int NS>
+struct FwdCfg {
+    static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along d
+    static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
+    static constexpr int kTileBytes = 128 * D * 2;      // a 128-row tile of Q, K or V
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + NQ * kTileBytes;
+    static constexpr int kVOff = kKOff + NS * kTileBytes;
+    static constexpr int kBarOff = kVOff + NS * kTileBytes;
+    // barrier indices
+    static constexpr int kBarQ = 0;
+    static constexpr int kBarKFull = 1;
+    static constexpr int kBarVFull = kBarKFull + NS;
+    static constexpr int kBarKEmpty = kBarVFull + NS;
+    static constexpr int kBarVEmpty = kBarKEmpty + NS;
+    static constexpr int kBarSFull = kBarVEmpty + NS;
+    static constexpr int kBarPFull = kBarSFull + NQ;
+    static constexpr int kBarOFull = kBarPFull + NQ;
+    static constexpr int kBarMmaDone = kBarOFull + NQ;
+    static constexpr int kNumBars = kBarMmaDone + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + slack for 1 KB alignment
+    static constexpr int kSoftmaxWarps = 4 * NQ;
+    static constexpr int kWarpTma = kSoftmaxWarps;
+    static constexpr int kWarpMma = kSoftmaxWarps + 1;
+    static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+    static constexpr int kOCol = 256;
+    static_assert(D == 64 || D == 128 || D == 256, "head dim");
+    static_assert(256 + NQ * D <= 512, "TMEM columns");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+// Bounded wait that ignores the abort flag: used only to drain this CTA's own
+// TMA loads / MMAs before it releases shared or tensor memory.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const unsigned long long t0 = globaltimer();
+    uint32_t it = 0;
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((++it & 31u) == 0 && globaltimer() - t0 > kTimeoutNs) {
+            atomicCAS(&g_dev_status, 0, kErrTimeout);
+            return;
+        }
+    }
+}
+
+template <int D, int NQ, int NS, bool BF16>
+__global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+    using C = FwdCfg<D, NQ, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    // causal: the heaviest query blocks start first
+    const int qp = (p.mode & kCausal) ? static_cast<int>(gridDim.y - 1 - blockIdx.y)
+                                      : static_cast<int>(blockIdx.y);
+    const int rb0 = qp * NQ;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::kBarQ), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(C::kBarKFull + s), 1);
+            mbar_init(bar(C::kBarVFull + s), 1);
+            mbar_init(bar(C::kBarKEmpty + s), 1);
+            mbar_init(bar(C::kBarVEmpty + s), 1);
+        }
+        for (int t = 0; t < NQ; ++t) {
+            mbar_init(bar(C::kBarSFull + t), 1);
+            mbar_init(bar(C::kBarPFull + t), 128);
+            mbar_init(bar(C::kBarOFull + t), 1);
+        }
+        mbar_init(bar(C::kBarMmaDone), 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == C::kWarpMma) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    if (warp == C::kWarpTma && lane == 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == C::kWarpTma) {
+        // ------------------------------------------------------------ producer
+        int nq_valid = 0;
+        for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
+            for (int t = 0; t < NQ; ++t) {
+                if (rb0 + t >= p.nqb) continue;
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
+                                bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
+            }
+        }
+        __syncwarp();
+        KvIter<NQ> it;
+        int j;
+        uint32_t f;
+        int nk = 0, nv = 0;   // loads issued
+        bool ok = true;
+        while (ok && it.next(p, rb0, j, f)) {
+            const int s = nk % NS;
+            const uint32_t ph = (nk / NS) & 1;
+            ok = wait_bar(bar(C::kBarKEmpty + s), ph ^ 1u, abort_flag);
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
+                                bar(C::kBarKFull + s), c * 64, j * 128, bh);
+            }
+            ++nk;
+            ok = wait_bar(bar(C::kBarVEmpty + s), ph ^ 1u, abort_flag);
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
+                                bar(C::kBarVFull + s), c * 64, j * 128, bh);
+            }
+            ++nv;
+            __syncwarp();
+        }
+        // every issued load has landed before the CTA may exit
+        drain_bar(bar(C::kBarQ), 0);
+        for (int i = (nk > NS ? nk - NS : 0); i < nk; ++i)
+            drain_bar(bar(C::kBarKFull + i % NS), (i / NS) & 1);
+        for (int i = (nv > NS ? nv - NS : 0); i < nv; ++i)
+            drain_bar(bar(C::kBarVFull + i % NS), (i / NS) & 1);
+    } else if (warp == C::kWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t kIdescS = instr_desc_f16(128, 128, BF16, false, false);
+        constexpr uint32_t kIdescO = instr_desc_f16(128, D, BF16, false, true);
+        auto issue_s = [&](int t, int s) {
+            const uint32_t a0 = sbase + C::kQOff + t * C::kTileBytes;
+            const uint32_t b0 = sbase + C::kKOff + s * C::kTileBytes;
+            const uint32_t d_tmem = tmem + 128u * t;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint32_t koff = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
+                mma_ss(d_tmem, smem_desc_sw128(a0 + koff, 16, 1024),
+                       smem_desc_sw128(b0 + koff, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_pv = [&](int t, int s, bool acc) {
+            const uint32_t b0 = sbase + C::kVOff + s * C::kTileBytes;
+            const uint32_t d_tmem = tmem + C::kOCol + D * t;
+            const uint32_t a_tmem = tmem + 128u * t;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                mma_ts(d_tmem, a_tmem + 8u * k, smem_desc_sw128(b0 + k * 2048, C::kChunkBytes, 1024),
+                       kIdescO, (acc || k > 0) ? 1u : 0u);
+        };
+
+        KvIter<NQ> it;
+        int j, jn;
+        uint32_t f, fn;
+        int cnt[NQ];
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) cnt[t] = 0;
+        bool have = it.next(p, rb0, j, f);
+        bool ok = true;
+        if (have) {
+            ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) {
+                    for (int t = 0; t < NQ; ++t)
+                        if ((f >> t) & 1u) {
+                            issue_s(t, 0);
+                            mma_commit(bar(C::kBarSFull + t));
+                        }
+                    mma_commit(bar(C::kBarKEmpty));
+                }
+                __syncwarp();
+            }
+        }
+        int u = 0;
+        while (ok && have) {
+            const int s = u % NS;
+            const uint32_t ph = (u / NS) & 1;
+            const bool have_n = it.next(p, rb0, jn, fn);
+            const int sn = (u + 1) % NS;
+            const uint32_t phn = ((u + 1) / NS) & 1;
+            ok = wait_bar(bar(C::kBarVFull + s), ph, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            bool k_ready = false;
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) {
+                if ((f >> t) & 1u) {
+                    ok = wait_bar(bar(C::kBarPFull + t), cnt[t] & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) issue_pv(t, s, cnt[t] > 0);
+                    __syncwarp();
+                    ++cnt[t];
+                }
+                if (have_n && ((fn >> t) & 1u)) {
+                    if (!k_ready) {
+                        ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        k_ready = true;
+                    }
+                    if (lane == 0) {
+                        issue_s(t, sn);
+                        mma_commit(bar(C::kBarSFull + t));
+                    }
+                    __syncwarp();
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                mma_commit(bar(C::kBarVEmpty + s));
+                if (have_n) mma_commit(bar(C::kBarKEmpty + sn));
+            }
+            __syncwarp();
+            j = jn;
+            f = fn;
+            have = have_n;
+            ++u;
+        }
+        if (lane == 0) {
+            for (int t = 0; t < NQ; ++t) mma_commit(bar(C::kBarOFull + t));
+            mma_commit(bar(C::kBarMmaDone));
+        }
+        __syncwarp();
+        drain_bar(bar(C::kBarMmaDone), 0);
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int t = warp >> 2;
+        const int wq = warp & 3;
+        const int rb = rb0 + t;
+        const int row_local = wq * 32 + lane;
+        const int row = rb * 128 + row_local;
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 128u * t;
+        const uint32_t tO = tmem + lane_off + C::kOCol + D * t;
+        const float c = p.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        int cnt = 0;
+        KvIter<NQ> it;
+        int j;
+        uint32_t f;
+        bool ok = true;
+        while (it.next(p, rb0, j, f)) {
+            if (!((f >> t) & 1u)) continue;
+            ok = wait_bar(bar(C::kBarSFull + t), cnt & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t r[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
+            tmem_ld_wait();
+            float sv[128];
+#pragma unroll
+            for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
+            const bool diag = (p.mode & kCausal) && j == rb;
+            const bool tail = (j == p.nkb - 1) && (p.N & 127);
+            if (diag || tail) {
+                int lim = tail ? (p.N - j * 128) : 128;
+                if (diag) lim = min(lim, row_local + 1);
+#pragma unroll
+                for (int k = 0; k < 128; ++k)
+                    if (k >= lim) sv[k] = -INFINITY;
+            }
+            float mx = sv[0];
+#pragma unroll
+            for (int k = 1; k < 128; ++k) mx = fmaxf(mx, sv[k]);
+            const float m_cand = fmaxf(m, mx * c);
+            const bool grow = m_cand > m + 8.0f;    // lazy: keep m unless it moves by > 2^8
+            const float m_new = grow ? m_cand : m;
+            const float alpha = grow ? ex2(m - m_new) : 1.0f;
+            const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
+            if (cnt > 0 && __any_sync(0xffffffffu, grow)) {
+                // S_t's completion implies the previous O_t += P V finished
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * q, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                    tmem_st32(tO + 32 * q, o);
+                }
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float p0 = ex2(fmaf(sv[32 * q + 2 * k], c, -m_use));
+                    const float p1 = ex2(fmaf(sv[32 * q + 2 * k + 1], c, -m_use));
+                    sum += p0 + p1;
+                    pk[k] = pack2<BF16>(p0, p1);
+                }
+                tmem_st16(tS + 16 * q, pk);
+            }
+            l = l * alpha + sum;
+            m = m_new;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarPFull + t));
+            ++cnt;
+        }
+        if (ok && cnt > 0) ok = wait_bar(bar(C::kBarOFull + t), 0, abort_flag);
+        tc_fence_after();
+        if (rb < p.nqb && ok) {
+            const bool valid = row < p.N;
+            const float inv_l = (cnt > 0 && l > 0.f) ? 1.0f / l : 0.0f;
+            uint8_t *orow = reinterpret_cast<uint8_t *>(p.o) +
+                            (static_cast<size_t>(bh) * p.N + (valid ? row : 0)) * D * 2;
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t o[32];
+                if (cnt > 0) {
+                    tmem_ld32(tO + 32 * q, o);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    pk[k] = pack2<BF16>(__uint_as_float(o[2 * k]) * inv_l,
+                                        __uint_as_float(o[2 * k + 1]) * inv_l);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 64);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                }
+            }
+            if (valid) {
+                const float lse = (cnt > 0 && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f
+                                                        : -INFINITY;
+                p.lse[static_cast<size_t>(bh) * p.N + row] = lse;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fa

@@ -1,0 +1,140 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library libfa_b200.so.
+ *
+ * Computes exact softmax attention O = softmax(scale * Q K^T [+ mask]) V
+ * ("FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness" notes, section 1.1) with the tiled online softmax of
+ * "FlashAttention 深度解析" section 二, so the N x N score and probability
+ * matrices never reach device memory ("FlashAttention原理概览" section 3.1).
+ * The forward saves one fp32 log-sum-exp per query row; the backward
+ * recomputes P from it ("原理概览" section 3.2; notes section 2.5).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout     q, k, v, o, dout, dq, dk, dv are contiguous [B][H][N][d] arrays
+ *            of 16-bit floats (d innermost); lse is contiguous fp32 [B][H][N].
+ *            All are DEVICE pointers on the current CUDA device.
+ * dtype      FA_F16 or FA_BF16, the element type of every 16-bit array.
+ *            Products accumulate in fp32; P is rounded to dtype before P.V
+ *            and outputs are rounded to nearest even.
+ * d          64, 128 or 256 (the head-dimension limit of "深度解析" section
+ *            五; a multiple of 16 per "原理概览" section 3.4).
+ * N          any N >= 1; a ragged last tile is masked.  N is both the query
+ *            and the key length.
+ * scale      the softmax scale, supplied by the caller (usually 1/sqrt(d)).
+ * causal     nonzero: query i sees key j only when j <= i ("深度解析" 五).
+ * stream     a cudaStream_t passed as void*; NULL means the legacy default
+ *            stream.  Every call is asynchronous on it.
+ * Ownership  the caller allocates and frees every buffer; the library
+ *            allocates no device memory.  Inputs are only read; outputs are
+ *            completely overwritten.  Buffers must not overlap.
+ * Alignment  every pointer must be 16-byte aligned, else FA_ERR_MISALIGNED.
+ * Errors     a non-zero fa_status; nothing is launched when the arguments
+ *            are rejected.  A failed launch returns FA_ERR_CUDA.  Kernels
+ *            bound every wait; one that gives up records FA_ERR_TIMEOUT in a
+ *            device word that fa_last_device_status() returns after the
+ *            caller has synchronised.
+ * Rows with no visible key (possible only with a hand-made block mask whose
+ * whole block row is zero) get O = 0, LSE = -inf and zero gradients.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad flag, non-finite scale */
+    FA_ERR_UNSUPPORTED = 2,  /* d not in {64, 128, 256}, or a size beyond the kernel limits */
+    FA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than fa_bwd_workspace_bytes() */
+    FA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+    FA_ERR_TIMEOUT = 6       /* a kernel gave up waiting (see fa_last_device_status) */
+} fa_status;
+
+/* Side length of one block-mask block, in rows and keys. */
+#define FA_BLOCK 128
+
+/*
+ * Forward pass.  Writes o [B][H][N][d] and lse [B][H][N] with
+ * lse_i = ln sum_j exp(scale * q_i . k_j) over the keys visible to row i
+ * (the row statistics m and l of "原理概览" section 3.2 folded into one
+ * natural-log value).
+ */
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int H, int N, int d, float scale, int causal, int dtype,
+                  void *stream);
+
+/*
+ * Block-sparse forward ("FlashAttention" notes, section 4): block_mask is a
+ * DEVICE uint8 array [nb][nb], nb = ceil(N / FA_BLOCK), row-major, shared by
+ * every (batch, head).  Query block r attends to key block c only when
+ * block_mask[r * nb + c] != 0; skipped blocks are never loaded or computed.
+ * causal may be combined with the mask (diagonal blocks then get the
+ * element-wise causal mask as well).
+ */
+FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const uint8_t *block_mask,
+                              int B, int H, int N, int d, float scale, int causal, int dtype,
+                              void *stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: an fp32 D = rowsum(dO * O) per row
+ * and an fp32 dQ accumulator [B][H][N][d].  Returns 0 for invalid sizes.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass ("深度解析" section 四: five matrix products; P recomputed
+ * from lse per "原理概览" section 3.2).  Reads q, k, v, o, dout and the lse
+ * written by fa_fwd with the same arguments; writes dq, dk, dv.  workspace is
+ * a caller-owned DEVICE buffer of at least fa_bwd_workspace_bytes() bytes,
+ * 16-byte aligned; its contents on entry do not matter and on exit are
+ * unspecified.  dq is accumulated with fp32 atomics, so its low bits may
+ * differ from run to run; dk and dv are deterministic.
+ */
+FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                  const float *lse, void *dq, void *dk, void *dv,
+                  void *workspace, size_t workspace_bytes,
+                  int B, int H, int N, int d, float scale, int causal, int dtype,
+                  void *stream);
+
+/* Block-sparse backward; block_mask as for fa_fwd_blocksparse. */
+FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
+                              const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                              void *workspace, size_t workspace_bytes,
+                              const uint8_t *block_mask,
+                              int B, int H, int N, int d, float scale, int causal, int dtype,
+                              void *stream);
+
+/* A static, human-readable name for a status code. */
+FA_API const char *fa_status_string(int status);
+
+/*
+ * The device error word written by kernels that gave up waiting
+ * (FA_ERR_TIMEOUT) since the last call, then cleared.  Synchronises the
+ * current device.  FA_OK when nothing went wrong.
+ */
+FA_API int fa_last_device_status(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

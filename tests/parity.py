@@ -1,0 +1,76 @@
+"""Shared helpers for the GPU parity tests: seeded inputs -> CUDA path (through
+the C ABI binding) and -> fp64 oracle, compared element by element.
+
+Tolerances (max absolute error unless stated):
+  O   1e-2 (fp16), 2e-2 (bf16)
+  LSE 1e-3
+  dQ, dK, dV  5e-2 * max |oracle value| of that tensor
+"""
+import numpy as np
+import torch
+
+import oracle
+from flash_fwd_b200 import inputs
+
+TOL_O = {"f16": 1e-2, "bf16": 2e-2}
+TOL_LSE = 1e-3
+TOL_GRAD_REL = 5e-2
+
+
+def bh(x):
+    """[B, H, N, d] -> float64 numpy [B*H, N, d]."""
+    return x.reshape(-1, x.shape[-2], x.shape[-1]).double().numpy()
+
+
+def flags(causal, mask):
+    return (oracle.CAUSAL if causal else 0) | (oracle.SPARSE if mask is not None else 0)
+
+
+def mask_np(mask):
+    return None if mask is None else mask.numpy().astype(np.uint8)
+
+
+def gpu_fwd(q, k, v, causal, scale, mask=None):
+    import flash_fwd_b200 as fa
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    md = mask.to(dev) if mask is not None else None
+    o, lse = fa.attention_fwd(qd, kd, vd, causal=causal, scale=scale, block_mask=md)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    return o.cpu(), lse.cpu()
+
+
+def gpu_bwd(q, k, v, o, do, lse, causal, scale, mask=None):
+    import flash_fwd_b200 as fa
+    dev = torch.device("cuda:0")
+    args = [t.to(dev) for t in (q, k, v, o, do)]
+    md = mask.to(dev) if mask is not None else None
+    dq, dk, dv = fa.attention_bwd(*args, lse.to(dev), causal=causal, scale=scale, block_mask=md)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def check_fwd(o_gpu, lse_gpu, q, k, v, causal, scale, dtype, mask=None, rows_per_head=None, seed=0):
+    """Compares O and LSE with the oracle on every row, or on sampled rows per head."""
+    B, H, N, d = q.shape
+    Q, K, V = bh(q), bh(k), bh(v)
+    og = o_gpu.reshape(B * H, N, d).double().numpy()
+    lg = lse_gpu.reshape(B * H, N).double().numpy()
+    worst_o, worst_l = 0.0, 0.0
+    if rows_per_head is None:
+        o_ref, l_ref = oracle.fwd(Q, K, V, scale, flags(causal, mask), mask_np(mask))
+        worst_o = np.abs(og - o_ref).max()
+        worst_l = np.abs(lg - l_ref).max()
+    else:
+        for h in range(B * H):
+            rows = inputs.sample_rows(N, rows_per_head, seed, h).numpy()
+            o_ref, l_ref = oracle.fwd_rows(Q[h:h + 1], K[h:h + 1], V[h:h + 1], scale, flags(causal, mask),
+                                           mask_np(mask), 128, rows)
+            worst_o = max(worst_o, np.abs(og[h, rows] - o_ref[0]).max())
+            worst_l = max(worst_l, np.abs(lg[h, rows] - l_ref[0]).max())
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    assert worst_o <= TOL_O[dtype], f"O max err {worst_o}"
+    assert worst_l <= TOL_LSE, f"LSE max err {worst_l}"
+    return worst_o, worst_l
