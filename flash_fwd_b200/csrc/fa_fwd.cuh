@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
         const uint32_t tS = tmem + lane_off + 128u * t;
         const uint32_t tO = tmem + lane_off + C::kOCol + D * t;
         const float c = p.scale_log2;
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f, l_r = 0.f;
         int cnt = 0;
         KvIter<NQ> it;
         int j;
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
                     tmem_st32(tO + 32 * q, o);
                 }
             }
-            float sum = 0.f;
+            float sum = 0.f, sum_r = 0.f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t pk[16];
@@ -393,12 +393,19 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
                 for (int k = 0; k < 16; ++k) {
                     const float p0 = ex2(fmaf(sv[32 * q + 2 * k], c, -m_use));
                     const float p1 = ex2(fmaf(sv[32 * q + 2 * k + 1], c, -m_use));
-                    sum += p0 + p1;
                     pk[k] = pack2<BF16>(p0, p1);
+                    sum += p0 + p1;
+                    if constexpr (BF16) {
+                        // O is normalised by the sum of the same rounded P the
+                        // tensor core multiplies (a row dominated by one key then
+                        // comes out exact); LSE keeps the unrounded sum
+                        sum_r += __uint_as_float(pk[k] << 16) + __uint_as_float(pk[k] & 0xffff0000u);
+                    }
                 }
                 tmem_st16(tS + 16 * q, pk);
             }
             l = l * alpha + sum;
+            if constexpr (BF16) l_r = l_r * alpha + sum_r;
             m = m_new;
             tmem_st_wait();
             tc_fence_before();
@@ -409,7 +416,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
         tc_fence_after();
         if (rb < p.nqb && ok) {
             const bool valid = row < p.N;
-            const float inv_l = (cnt > 0 && l > 0.f) ? 1.0f / l : 0.0f;
+            const float l_o = BF16 ? l_r : l;
+            const float inv_l = (cnt > 0 && l_o > 0.f) ? 1.0f / l_o : 0.0f;
             uint8_t *orow = reinterpret_cast<uint8_t *>(p.o) +
                             (static_cast<size_t>(bh) * p.N + (valid ? row : 0)) * D * 2;
 #pragma unroll 1
