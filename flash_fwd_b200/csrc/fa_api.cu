@@ -111,6 +111,101 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
                             : dispatch_fwd<false>(d, mq, mk, mv, p, BH, s);
 }
 
+
+template <int D, int BM, int DSPLIT, int NS, bool DQT, bool BF16>
+int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+               void *dq, void *dk, void *dv, float *dvec, float *dqacc, const uint8_t *mask, int BH, int N,
+               float scale, int causal, int dtype, cudaStream_t stream) {
+    using C = fa::BwdCfg<D, BM, DSPLIT, NS, DQT>;
+    const long long rows = static_cast<long long>(BH) * N;
+    // D = rowsum(dO o O) and dQacc = 0
+    {
+        constexpr int TPR = D / 8;
+        const long long threads = rows * TPR;
+        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        fa::bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), dvec, reinterpret_cast<float4 *>(dqacc),
+            rows);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    CUtensorMap mk, mv, mq, mdo;
+    int rc;
+    if ((rc = make_map(&mk, k, D, N, BH, dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, D, N, BH, dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, q, D, N, BH, dtype, BM)) != FA_OK) return rc;
+    if ((rc = make_map(&mdo, dout, D, N, BH, dtype, BM)) != FA_OK) return rc;
+    fa::BwdParams p;
+    p.lse = lse;
+    p.dvec = dvec;
+    p.dqacc = dqacc;
+    p.dk = dk;
+    p.dv = dv;
+    p.mask = mask;
+    p.N = N;
+    p.nkb = (N + 127) / 128;
+    p.nqt = (N + BM - 1) / BM;
+    p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    auto kern = fa::bwd_kernel<D, BM, DSPLIT, NS, DQT, BF16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    dim3 grid(p.nkb * DSPLIT, BH);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    // dQ = scale * dQacc
+    {
+        const long long n8 = rows * D / 8;
+        const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+        fa::bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dqacc),
+                                                               static_cast<uint4 *>(dq), scale, n8);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
+template <bool BF16>
+int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, float *dvec, float *dqacc, const uint8_t *mask,
+                 int BH, int N, float scale, int causal, int dtype, cudaStream_t s) {
+    switch (d) {
+        case 64:
+            return launch_bwd<64, 128, 1, 3, false, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+                                                          N, scale, causal, dtype, s);
+        case 128:
+            return launch_bwd<128, 64, 1, 3, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+                                                         N, scale, causal, dtype, s);
+        case 256:
+            return launch_bwd<256, 64, 2, 1, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+                                                         N, scale, causal, dtype, s);
+        default: return FA_ERR_UNSUPPORTED;
+    }
+}
+
+int bwd_impl(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+             void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, const uint8_t *mask, int B,
+             int H, int N, int d, float scale, int causal, int dtype, void *stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    const void *ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+    const long long BH = static_cast<long long>(B) * H;
+    const size_t need = fa::bwd_workspace_bytes(BH, N, d);
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+    float *dvec = static_cast<float *>(workspace);
+    float *dqacc = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                             ((static_cast<size_t>(BH) * N * 4 + 255) & ~static_cast<size_t>(255)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dtype == FA_BF16
+               ? dispatch_bwd<true>(d, q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, static_cast<int>(BH), N,
+                                    scale, causal, dtype, s)
+               : dispatch_bwd<false>(d, q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, static_cast<int>(BH),
+                                     N, scale, causal, dtype, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -135,8 +230,8 @@ FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
                   void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int N,
                   int d, float scale, int causal, int dtype, void *stream) {
-    return fa::bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d,
-                         scale, causal, dtype, stream);
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d, scale,
+                    causal, dtype, stream);
 }
 
 FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const void *dout,
@@ -144,8 +239,8 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, const uint8_t *block_mask, int B, int H, int N, int d,
                               float scale, int causal, int dtype, void *stream) {
     if (!block_mask) return FA_ERR_INVALID_ARG;
-    return fa::bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, block_mask, B, H, N,
-                         d, scale, causal, dtype, stream);
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, block_mask, B, H, N, d, scale,
+                    causal, dtype, stream);
 }
 
 FA_API const char *fa_status_string(int status) {

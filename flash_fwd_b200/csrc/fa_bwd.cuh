@@ -1,14 +1,542 @@
-// fa_bwd.cuh -- backward kernels (placeholder until the kernels land).
+// fa_bwd.cuh -- backward kernels of exact attention for sm_100a.
+//
+// What is computed (per (batch, head); "FlashAttention 深度解析" section 四:
+// five matrix products; "FlashAttention原理概览" section 3.2: P is recomputed
+// from the saved row statistics instead of being stored):
+//   P  = exp(scale * Q K^T - LSE)          (recomputed, never stored)
+//   dV = P^T dO,   dP = dO V^T,   D_i = sum_c dO_ic O_ic,
+//   dS = P o (dP - D),   dQ = scale * dS K,   dK = scale * dS^T Q.
+//
+// Three launches on the caller's stream:
+//   bwd_pre   D = rowsum(dO o O) into the workspace; zeroes the fp32 dQ accumulator.
+//   bwd_main  one CTA per 128-key block (x DSPLIT column halves for d = 256).  The
+//             CTA keeps K_j, V_j in shared memory and its dK, dV accumulators in
+//             tensor memory while it sweeps the kept query tiles Q_i, dO_i
+//             (BM rows each) through an NS-stage TMA ring:
+//               S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T   (tcgen05, TMEM)
+//               P^T, dS^T          (softmax-grad warps, one thread per key row,
+//                                   written as 16-bit swizzled tiles to smem)
+//               dV  += P^T dO_i,   dK += dS^T Q_i        (tcgen05, TMEM)
+//               dQ_i = dS K_j  (d = 64)  or  dQ_i^T = K_j^T dS^T  (d >= 128)
+//                                  (tcgen05, TMEM), then fp32 atomics into the
+//                                   accumulator by the drain warps.
+//   bwd_post  dQ = scale * accumulator, rounded to the 16-bit type.
+//
+// Warp roles of bwd_main: warps 0-3 softmax-grad (and the dV epilogue), warps
+// 4-7 dQ drain (and the dK epilogue), warp 8 TMA producer (also stages the
+// per-row LSE and D of each query tile), warp 9 MMA issuer (owns TMEM).
+// TMEM columns: S^T [0, BM), dP^T [128, 128 + BM), dV [256, 256 + DH),
+// dK [256 + DH, 256 + 2 DH), dQ at [64, 128) (transposed form) or
+// [256 + 2 DH, 256 + 3 DH) (d = 64).
 #pragma once
+
 #include "fa_common.cuh"
-#include "fa.h"
+#include "fa_fwd.cuh"
 
 namespace fa {
+
+struct BwdParams {
+    const float *lse;     // [BH][N] natural-log LSE from the forward
+    const float *dvec;    // [BH][N] D = rowsum(dO o O)
+    float *dqacc;         // [BH][N][D] fp32, zeroed by bwd_pre
+    void *dk;             // [BH][N][D] 16-bit
+    void *dv;             // [BH][N][D] 16-bit
+    const uint8_t *mask;  // [nkb][nkb] block mask (kSparse)
+    int N;
+    int nkb;              // key blocks (and mask blocks) of 128
+    int nqt;              // query tiles of BM rows
+    int mode;
+    float scale;
+    float scale_log2;
+};
+
+// ---------------------------------------------------------------------------
+// bwd_pre: D_i = sum_c dO_ic O_ic, and dQacc = 0
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint4 *__restrict__ o, const uint4 *__restrict__ dout,
+                                                      float *__restrict__ dvec, float4 *__restrict__ dqacc,
+                                                      long long rows) {
+    constexpr int TPR = D / 8;   // threads per row, 8 elements (16 bytes) each
+    const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long row = tid / TPR;
+    const int part = static_cast<int>(tid % TPR);
+    float acc = 0.f;
+    if (row < rows) {
+        const uint4 a = o[row * TPR + part];
+        const uint4 b = dout[row * TPR + part];
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 x = unpack2<BF16>(av[k]), y = unpack2<BF16>(bv[k]);
+            acc = fmaf(x.x, y.x, acc);
+            acc = fmaf(x.y, y.y, acc);
+        }
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        dqacc[(row * D + part * 8) / 4] = z;
+        dqacc[(row * D + part * 8) / 4 + 1] = z;
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) dvec[row] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// bwd_post: dQ = scale * dQacc in the 16-bit type
+// ---------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict__ acc, uint4 *__restrict__ dq,
+                                                       float scale, long long n8) {
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = acc[2 * i], b = acc[2 * i + 1];
+    dq[i] = make_uint4(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale),
+                       pack2<BF16>(b.x * scale, b.y * scale), pack2<BF16>(b.z * scale, b.w * scale));
+}
+
+// ---------------------------------------------------------------------------
+// bwd_main
+// ---------------------------------------------------------------------------
+template <int BM>
+__device__ __forceinline__ bool qtile_kept(const BwdParams &p, int i, int j) {
+    if (i >= p.nqt) return false;
+    if ((p.mode & kCausal) && (i + 1) * BM <= j * 128) return false;   // every query precedes every key
+    if ((p.mode & kSparse) && p.mask[static_cast<size_t>((i * BM) / 128) * p.nkb + j] == 0) return false;
+    return true;
+}
+
+// Walks the query tiles that see key block j, in increasing order (warp-collective).
+template <int BM>
+struct QIter {
+    int base = -32;
+    uint32_t b = 0;
+    __device__ __forceinline__ bool next(const BwdParams &p, int j, int &i) {
+        while (b == 0u) {
+            base += 32;
+            if (base >= p.nqt) return false;
+            b = __ballot_sync(0xffffffffu, qtile_kept<BM>(p, base + static_cast<int>(lane_id()), j));
+        }
+        const int k = __ffs(b) - 1;
+        b &= b - 1;
+        i = base + k;
+        return true;
+    }
+};
+
+template <int D, int BM, int DSPLIT, int NS, bool DQT>
+struct BwdCfg {
+    static constexpr int DH = D / DSPLIT;                 // output columns per CTA
+    static constexpr int kKVTile = 128 * D * 2;           // K_j or V_j
+    static constexpr int kKVChunk = 128 * 128;            // 64 columns of a 128-row tile
+    static constexpr int kQTile = BM * D * 2;             // Q_i or dO_i
+    static constexpr int kQChunk = BM * 128;              // 64 columns of a BM-row tile
+    static constexpr int kPTile = 128 * BM * 2;           // P^T or dS^T: 128 keys x BM queries
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kKVTile;
+    static constexpr int kQOff = kVOff + kKVTile;
+    static constexpr int kdOOff = kQOff + NS * kQTile;
+    static constexpr int kPOff = kdOOff + NS * kQTile;
+    static constexpr int kdSOff = kPOff + kPTile;
+    static constexpr int kStatOff = kdSOff + kPTile;      // per stage: lse*log2e [BM], D [BM]
+    static constexpr int kBarOff = kStatOff + NS * BM * 8;
+    static constexpr int kBarKV = 0;
+    static constexpr int kBarQFull = 1;
+    static constexpr int kBarQEmpty = kBarQFull + NS;
+    static constexpr int kBarSdpFull = kBarQEmpty + NS;
+    static constexpr int kBarSdpEmpty = kBarSdpFull + 1;
+    static constexpr int kBarDsFull = kBarSdpEmpty + 1;
+    static constexpr int kBarPdsEmpty = kBarDsFull + 1;
+    static constexpr int kBarDqFull = kBarPdsEmpty + 1;
+    static constexpr int kBarDqEmpty = kBarDqFull + 1;
+    static constexpr int kBarMmaDone = kBarDqEmpty + 1;
+    static constexpr int kNumBars = kBarMmaDone + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+    static constexpr int kThreads = 320;
+    static constexpr int kColS = 0;
+    static constexpr int kColDP = 128;
+    static constexpr int kColDV = 256;
+    static constexpr int kColDK = 256 + DH;
+    static constexpr int kColDQ = DQT ? 64 : 256 + 2 * DH;
+    static constexpr int kDqCols = DQT ? BM : DH;         // fp32 columns per drain thread
+    static_assert(DQT ? (BM == 64 && DH == 128) : (BM == 128 && DH == 64), "tile shape");
+    static_assert(kColDQ + kDqCols <= 512 && kColDK + DH <= 512, "TMEM columns");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+template <int D, int BM, int DSPLIT, int NS, bool DQT, bool BF16>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+               const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
+               const BwdParams p) {
+    using C = BwdCfg<D, BM, DSPLIT, NS, DQT>;
+    constexpr int DH = C::DH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x / DSPLIT;
+    const int h = blockIdx.x % DSPLIT;
+    const int bh = blockIdx.y;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::kBarKV), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(C::kBarQFull + s), 1);
+            mbar_init(bar(C::kBarQEmpty + s), 1);
+        }
+        mbar_init(bar(C::kBarSdpFull), 1);
+        mbar_init(bar(C::kBarSdpEmpty), 128);
+        mbar_init(bar(C::kBarDsFull), 128);
+        mbar_init(bar(C::kBarPdsEmpty), 1);
+        mbar_init(bar(C::kBarDqFull), 1);
+        mbar_init(bar(C::kBarDqEmpty), 128);
+        mbar_init(bar(C::kBarMmaDone), 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmdo);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    int cnt = 0;        // query tiles processed by this warp's role
+    bool ok = true;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVTile);
+            for (int c = 0; c < D / 64; ++c) {
+                tma_load_3d(sbase + C::kKOff + c * C::kKVChunk, &tmk, bar(C::kBarKV), c * 64, j * 128, bh);
+                tma_load_3d(sbase + C::kVOff + c * C::kKVChunk, &tmv, bar(C::kBarKV), c * 64, j * 128, bh);
+            }
+        }
+        __syncwarp();
+        QIter<BM> it;
+        int i;
+        while (it.next(p, j, i)) {
+            const int s = cnt % NS;
+            const uint32_t ph = (cnt / NS) & 1;
+            ok = wait_bar(bar(C::kBarQEmpty + s), ph ^ 1u, abort_flag);
+            if (!ok) break;
+            float *st = reinterpret_cast<float *>(smem + C::kStatOff + s * BM * 8);
+            for (int k = lane; k < BM; k += 32) {
+                const int q = i * BM + k;
+                float l2 = INFINITY, dd = 0.f;     // rows past N (or with no visible key) give P = 0
+                if (q < p.N) {
+                    const float L = p.lse[static_cast<size_t>(bh) * p.N + q];
+                    if (L != -INFINITY) l2 = L * 1.4426950408889634f;
+                    dd = p.dvec[static_cast<size_t>(bh) * p.N + q];
+                }
+                st[k] = l2;
+                st[BM + k] = dd;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(C::kBarQFull + s), 2 * C::kQTile);
+                for (int c = 0; c < D / 64; ++c) {
+                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, bar(C::kBarQFull + s),
+                                c * 64, i * BM, bh);
+                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo,
+                                bar(C::kBarQFull + s), c * 64, i * BM, bh);
+                }
+            }
+            __syncwarp();
+            ++cnt;
+        }
+        drain_bar(bar(C::kBarKV), 0);
+        for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t kIdS = instr_desc_f16(128, BM, BF16, false, false);
+        constexpr uint32_t kIdKV = instr_desc_f16(128, DH, BF16, false, true);
+        constexpr uint32_t kIdQ = DQT ? instr_desc_f16(128, BM, BF16, true, true)
+                                      : instr_desc_f16(128, DH, BF16, true, true);
+        const uint32_t sK = sbase + C::kKOff, sV = sbase + C::kVOff;
+        const uint32_t sP = sbase + C::kPOff, sdS = sbase + C::kdSOff;
+        auto issue_sdp = [&](int s) {
+            const uint32_t sQ = sbase + C::kQOff + s * C::kQTile, sdO = sbase + C::kdOOff + s * C::kQTile;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
+                const uint32_t oq = (k >> 2) * C::kQChunk + (k & 3) * 32;
+                mma_ss(tmem + C::kColS, smem_desc_sw128(sK + okv, 16, 1024), smem_desc_sw128(sQ + oq, 16, 1024),
+                       kIdS, k > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
+                const uint32_t oq = (k >> 2) * C::kQChunk + (k & 3) * 32;
+                mma_ss(tmem + C::kColDP, smem_desc_sw128(sV + okv, 16, 1024),
+                       smem_desc_sw128(sdO + oq, 16, 1024), kIdS, k > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_dvdk = [&](int s, bool acc) {
+            const uint32_t sQ = sbase + C::kQOff + s * C::kQTile, sdO = sbase + C::kdOOff + s * C::kQTile;
+            const uint32_t half = h * (DH / 64) * C::kQChunk;
+#pragma unroll
+            for (int k = 0; k < BM / 16; ++k) {
+                const uint32_t oa = (k >> 2) * (128 * 128) + (k & 3) * 32;
+                mma_ss(tmem + C::kColDV, smem_desc_sw128(sP + oa, 16, 1024),
+                       smem_desc_sw128(sdO + half + k * 2048, C::kQChunk, 1024), kIdKV, (acc || k > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < BM / 16; ++k) {
+                const uint32_t oa = (k >> 2) * (128 * 128) + (k & 3) * 32;
+                mma_ss(tmem + C::kColDK, smem_desc_sw128(sdS + oa, 16, 1024),
+                       smem_desc_sw128(sQ + half + k * 2048, C::kQChunk, 1024), kIdKV, (acc || k > 0) ? 1u : 0u);
+            }
+        };
+        auto issue_dq = [&]() {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if constexpr (DQT) {
+                    // dQ^T (DH x BM) = K_j^T (DH x 128 keys) * dS^T (128 keys x BM)
+                    mma_ss(tmem + C::kColDQ,
+                           smem_desc_sw128(sK + h * (DH / 64) * C::kKVChunk + k * 2048, C::kKVChunk, 1024),
+                           smem_desc_sw128(sdS + k * 2048, 128 * 128, 1024), kIdQ, k > 0 ? 1u : 0u);
+                } else {
+                    // dQ (BM x DH) = dS (BM x 128 keys) * K_j (128 keys x DH)
+                    mma_ss(tmem + C::kColDQ, smem_desc_sw128(sdS + k * 2048, 128 * 128, 1024),
+                           smem_desc_sw128(sK + k * 2048, C::kKVChunk, 1024), kIdQ, k > 0 ? 1u : 0u);
+                }
+            }
+        };
+
+        QIter<BM> it;
+        int i, in;
+        bool have = it.next(p, j, i);
+        if (have) {
+            ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_sdp(0);
+                    mma_commit(bar(C::kBarSdpFull));
+                }
+                __syncwarp();
+            }
+        }
+        // S^T, dP^T of the next tile: needs the softmax-grad warps to have read
+        // this tile's and the producer to have landed the next Q_i, dO_i
+        auto prefetch_next = [&]() -> bool {
+            const int sn = (cnt + 1) % NS;
+            if (!(wait_bar(bar(C::kBarSdpEmpty), cnt & 1, abort_flag) &&
+                  wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag)))
+                return false;
+            tc_fence_after();
+            if (lane == 0) {
+                issue_sdp(sn);
+                mma_commit(bar(C::kBarSdpFull));
+            }
+            __syncwarp();
+            return true;
+        };
+        while (ok && have) {
+            const int s = cnt % NS;
+            const bool have_n = it.next(p, j, in);
+            // with two or more stages the next tile is already resident: overlap
+            // its S^T, dP^T with this tile's softmax-grad work.  With one stage
+            // the next tile can only land after this tile's products finish.
+            if (NS >= 2 && have_n) {
+                ok = prefetch_next();
+                if (!ok) break;
+            }
+            ok = wait_bar(bar(C::kBarDsFull), cnt & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) issue_dvdk(s, cnt > 0);
+            __syncwarp();
+            ok = wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                issue_dq();
+                mma_commit(bar(C::kBarDqFull));
+                mma_commit(bar(C::kBarPdsEmpty));
+                mma_commit(bar(C::kBarQEmpty + s));
+            }
+            __syncwarp();
+            if (NS == 1 && have_n) {
+                ok = prefetch_next();
+                if (!ok) break;
+            }
+            ++cnt;
+            have = have_n;
+            i = in;
+        }
+        if (lane == 0) mma_commit(bar(C::kBarMmaDone));
+        __syncwarp();
+        drain_bar(bar(C::kBarMmaDone), 0);
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ softmax-grad
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const int r = warp * 32 + lane;     // key row within the block
+        const int key = j * 128 + r;
+        const float c = p.scale_log2;
+        uint8_t *sP = smem + C::kPOff;
+        uint8_t *sdS = smem + C::kdSOff;
+        QIter<BM> it;
+        int i;
+        while (it.next(p, j, i)) {
+            const int s = cnt % NS;
+            ok = wait_bar(bar(C::kBarSdpFull), cnt & 1, abort_flag) &&
+                 wait_bar(bar(C::kBarQFull + s), (cnt / NS) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const float *lse2 = reinterpret_cast<const float *>(smem + C::kStatOff + s * BM * 8);
+            const float *dd = lse2 + BM;
+            const bool need_causal = (p.mode & kCausal) && (i * BM < j * 128 + 127);
+#pragma unroll 1
+            for (int ch = 0; ch < BM / 32; ++ch) {
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tmem + lane_off + C::kColS + 32 * ch, sr);
+                tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, pr);
+                tmem_ld_wait();
+                if (ch == BM / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarSdpEmpty));
+                }
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    float pp[2], ds[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = 32 * ch + 2 * k + e;
+                        float pv = ex2(fmaf(__uint_as_float(sr[2 * k + e]), c, -lse2[col]));
+                        if (need_causal && key > i * BM + col) pv = 0.f;
+                        pp[e] = pv;
+                        ds[e] = pv * (__uint_as_float(pr[2 * k + e]) - dd[col]);
+                    }
+                    pk[k] = pack2<BF16>(pp[0], pp[1]);
+                    dk[k] = pack2<BF16>(ds[0], ds[1]);
+                }
+                if (ch == 0 && cnt > 0) {
+                    // the previous tile's dV/dK/dQ products must be done reading P^T, dS^T
+                    if (!wait_bar(bar(C::kBarPdsEmpty), (cnt - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                // row r of a K-major [BM/64][128][64] 128B-swizzled tile
+                const int chunk = (32 * ch) / 64;
+                const int u0 = ((32 * ch) % 64) / 8;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int off = chunk * (128 * 128) + r * 128 + (((u0 + u) ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(sP + off) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    *reinterpret_cast<uint4 *>(sdS + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+                }
+            }
+            if (!ok) break;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(bar(C::kBarDsFull));
+            ++cnt;
+        }
+    } else {
+        // ------------------------------------------------------------ dQ drain
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const int t = (warp & 3) * 32 + lane;   // TMEM lane: a d index (transposed form) or a query row
+        QIter<BM> it;
+        int i;
+        while (it.next(p, j, i)) {
+            ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[C::kDqCols];
+#pragma unroll
+            for (int ch = 0; ch < C::kDqCols / 32; ++ch)
+                tmem_ld32(tmem + lane_off + C::kColDQ + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarDqEmpty));
+            float *accb = p.dqacc + static_cast<size_t>(bh) * p.N * D;
+            if constexpr (DQT) {
+                const int dcol = h * DH + t;
+#pragma unroll
+                for (int k = 0; k < BM; ++k) {
+                    const int q = i * BM + k;
+                    if (q < p.N) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
+                }
+            } else {
+                const int q = i * BM + t;
+                if (q < p.N) {
+                    float4 *dst = reinterpret_cast<float4 *>(accb + static_cast<size_t>(q) * D + h * DH);
+#pragma unroll
+                    for (int k = 0; k < DH / 4; ++k)
+                        atomicAdd(dst + k, make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
+                }
+            }
+            ++cnt;
+        }
+    }
+
+    // ---------------------------------------------------------------- dV / dK epilogue
+    if (warp < 8) {
+        bool done = ok;
+        if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
+        tc_fence_after();
+        const bool is_dv = warp < 4;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const int r = (warp & 3) * 32 + lane;
+        const int key = j * 128 + r;
+        const float mul = is_dv ? 1.0f : p.scale;
+        uint8_t *out = reinterpret_cast<uint8_t *>(is_dv ? p.dv : p.dk);
+        const uint32_t col0 = is_dv ? C::kColDV : C::kColDK;
+        if (done) {
+#pragma unroll 1
+            for (int ch = 0; ch < DH / 32; ++ch) {
+                uint32_t v[32];
+                if (cnt > 0) {
+                    tmem_ld32(tmem + lane_off + col0 + 32 * ch, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] = 0u;
+                }
+                if (key < p.N) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D +
+                                                                  h * DH + 32 * ch) * 2);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 inline size_t bwd_workspace_bytes(long long BH, int N, int d) {
-    return static_cast<size_t>(BH) * N * 4 + static_cast<size_t>(BH) * N * d * 4 + 256;
+    const size_t dbytes = (static_cast<size_t>(BH) * N * 4 + 255) & ~static_cast<size_t>(255);
+    return dbytes + static_cast<size_t>(BH) * N * d * 4;
 }
-inline int bwd_entry(const void *, const void *, const void *, const void *, const void *, const float *, void *,
-                     void *, void *, void *, size_t, const uint8_t *, int, int, int, int, float, int, int, void *) {
-    return FA_ERR_UNSUPPORTED;
-}
+
 }  // namespace fa
