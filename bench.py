@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of exact attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch of synthetic input:
+fa_fwd (O, LSE) then fa_bwd (dQ, dK, dV), called through the C ABI.
+Throughput is TFLOP/s with the FLOP convention forward = 4*B*H*N^2*d (halved
+for causal), backward = 2.5 x forward; block-sparse counts kept blocks only.
+
+Default workload: B=4, H=16, N=4096, d=128, bf16, causal -- the shape on which
+the forward >= 60% / backward >= 45% of dense bf16 peak targets are quoted.
+
+With N > 1 (torchrun) every rank runs its own replica of the workload (weak
+scaling; the path needs no exchange step), timed on the device, max over ranks.
+
+Printed: one JSON line on rank 0 with value, roofline of the dominant kernel
+(CUDA events around each launch, recorded by the library on the launching
+stream), the CPU oracle baseline on a bounded sample (rank 0, N = 1 only), an
+end-to-end figure through host buffers, the SM clocks sampled during the timed
+region and the number of library kernel launches.
+
+--impl reference times the fp64 CPU oracle (the reference arm; there is no
+reference GPU code) on bounded samples of the same workload.
+"""
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPs/s at N=1K–64K, d=64–256; % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+
+WORKLOADS = {
+    "dsweep128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True),
+    "dsweep64": dict(B=4, H=16, N=4096, d=64, dtype="bf16", causal=True, sparse=False, bwd=True),
+    "dsweep256": dict(B=4, H=16, N=4096, d=256, dtype="bf16", causal=True, sparse=False, bwd=True),
+    "gpt2s": dict(B=8, H=12, N=1024, d=64, dtype="bf16", causal=True, sparse=False, bwd=True),
+    "long_fwd": dict(B=1, H=8, N=8192, d=128, dtype="f16", causal=False, sparse=False, bwd=False),
+    "long_fwd_causal": dict(B=1, H=8, N=8192, d=128, dtype="f16", causal=True, sparse=False, bwd=False),
+    "sparse64k": dict(B=1, H=4, N=65536, d=64, dtype="bf16", causal=False, sparse=True, bwd=True,
+                      density=0.2),
+    "tiny": dict(B=1, H=2, N=128, d=64, dtype="f16", causal=False, sparse=False, bwd=True),
+}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="dsweep128", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="wall-clock budget of the CPU oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("bf16_tflops"), p.get("bf16_tflops_sustained"), p.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def workload_flops(w, kept_blocks=None):
+    from flash_fwd_b200 import accounting as acc
+    if w["sparse"]:
+        f = acc.sparse_fwd_flops(w["B"], w["H"], w["d"], kept_blocks)
+    else:
+        f = acc.fwd_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
+    b = 2.5 * f if w["bwd"] else 0.0
+    return f, b
+
+
+def describe(name, w):
+    s = f"{name}: B={w['B']} H={w['H']} N={w['N']} d={w['d']} {w['dtype']}"
+    s += " causal" if w["causal"] else ""
+    s += f" block-sparse(128x128, diag + Bernoulli {w['density']})" if w["sparse"] else ""
+    s += " fwd+bwd" if w["bwd"] else " fwd"
+    return s
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "flash_fwd_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources are unchanged since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            lines = [ln.strip() for ln in f if ln.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_inputs(w, seed, device):
+    import torch
+
+    from flash_fwd_b200 import inputs
+    q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=seed, with_dout=w["bwd"])
+    mask = inputs.make_block_mask(w["N"], 128, w.get("density", 0.2), seed=seed) if w["sparse"] else None
+    host = dict(q=q, k=k, v=v, do=do, mask=mask)
+    dev = {n: (t.to(device) if t is not None else None) for n, t in host.items()}
+    dev["o"] = torch.empty_like(dev["q"])
+    dev["lse"] = torch.empty((w["B"], w["H"], w["N"]), dtype=torch.float32, device=device)
+    if w["bwd"]:
+        import flash_fwd_b200 as fa
+        dev["dq"], dev["dk"], dev["dv"] = (torch.empty_like(dev["q"]) for _ in range(3))
+        dev["ws"] = torch.empty(fa.fa_bwd_workspace_bytes(w["B"], w["H"], w["N"], w["d"]), dtype=torch.uint8,
+                                device=device)
+    return host, dev
+
+
+def step(w, t, stream):
+    import flash_fwd_b200 as fa
+    scale = 1.0 / w["d"] ** 0.5
+    if w["sparse"]:
+        fa.fa_fwd_blocksparse(t["q"], t["k"], t["v"], t["o"], t["lse"], t["mask"], w["causal"], scale, stream)
+        if w["bwd"]:
+            fa.fa_bwd_blocksparse(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"],
+                                  t["ws"], t["mask"], w["causal"], scale, stream)
+    else:
+        fa.fa_fwd(t["q"], t["k"], t["v"], t["o"], t["lse"], w["causal"], scale, stream)
+        if w["bwd"]:
+            fa.fa_bwd(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"], t["ws"],
+                      w["causal"], scale, stream)
+
+
+# --------------------------------------------------------------------------
+# CPU oracle: the baseline leg and the reference arm
+# --------------------------------------------------------------------------
+def oracle_head_pass(host, w, head):
+    """One (batch, head) of the workload through the fp64 oracle: forward on
+    every row, dQ on every row, dK/dV on every key.  Returns seconds."""
+    import numpy as np
+
+    import oracle
+    N, d = w["N"], w["d"]
+    b, h = divmod(head, w["H"])
+    sl = lambda t: t[b, h].reshape(1, N, d).double().numpy()  # noqa: E731
+    Q, K, V = sl(host["q"]), sl(host["k"]), sl(host["v"])
+    flags = (oracle.CAUSAL if w["causal"] else 0) | (oracle.SPARSE if w["sparse"] else 0)
+    mask = host["mask"].numpy() if w["sparse"] else None
+    rows = np.arange(N, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.fwd_rows(Q, K, V, 1.0 / d ** 0.5, flags, mask, 128, rows)
+    if w["bwd"]:
+        DO = sl(host["do"])
+        oracle.bwd_dq_rows(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128)
+        oracle.bwd_dkdv_cols(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128)
+    return time.perf_counter() - t0
+
+
+def per_head_flops(w, kept_blocks):
+    f, b = workload_flops(w, kept_blocks)
+    return (f + b) / (w["B"] * w["H"])
+
+
+def cpu_sample(host, w, kept_blocks, budget_s, max_heads=None):
+    heads = w["B"] * w["H"] if max_heads is None else min(max_heads, w["B"] * w["H"])
+    done, secs = 0, 0.0
+    while done < heads and (secs < budget_s or done == 0):
+        secs += oracle_head_pass(host, w, done)
+        done += 1
+    return done, secs, done * per_head_flops(w, kept_blocks) / secs / 1e12
+
+
+def run_reference(args, w, name):
+    from flash_fwd_b200 import dist as fdist
+    rank, world, _ = fdist.env_ranks()
+    if rank != 0:
+        return
+    host, _ = make_inputs_cpu(w)
+    kept = int(host["mask"].sum()) if w["sparse"] else None
+    for i in range(args.warmup):
+        oracle_head_pass(host, w, i % (w["B"] * w["H"]))
+    secs = 0.0
+    for i in range(args.steps):
+        secs += oracle_head_pass(host, w, (args.warmup + i) % (w["B"] * w["H"]))
+    val = args.steps * per_head_flops(w, kept) / secs / 1e12
+    cores = os.cpu_count()
+    sample = f"one (batch, head) of the workload per step: forward on all {w['N']} rows, dQ on all rows, dK/dV on all keys"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(name, w), "per_step": "one (batch, head)"},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def make_inputs_cpu(w):
+    from flash_fwd_b200 import inputs
+    q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=0, with_dout=w["bwd"])
+    mask = inputs.make_block_mask(w["N"], 128, w.get("density", 0.2), seed=0) if w["sparse"] else None
+    return dict(q=q, k=k, v=v, do=do, mask=mask), None
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args, w, name):
+    import torch
+
+    import flash_fwd_b200 as fa
+    from flash_fwd_b200 import dist as fdist
+
+    rank, world, local = fdist.init("nccl" if args.gpus > 1 else "gloo")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(device)
+    host, t = make_inputs(w, seed=rank, device=device)
+    kept = int(host["mask"].sum()) if w["sparse"] else None
+    fwd_f, bwd_f = workload_flops(w, kept)
+    flops = fwd_f + bwd_f
+
+    for _ in range(args.warmup):
+        step(w, t, stream)
+    torch.cuda.synchronize(device)
+    if fa.fa_last_device_status() != 0:
+        raise RuntimeError("device status after warm-up is not ok")
+
+    # ---------------- timed region: K steps on the device
+    sampler = ClockSampler(local)
+    fa.fa_profile_enable(True)
+    fa.fa_profile_read()
+    fdist.barrier(device)
+    torch.cuda.synchronize(device)
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(w, t, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    fdist.barrier(device)
+    clocks = sampler.stop()
+    prof = fa.fa_profile_read()
+    fa.fa_profile_enable(False)
+    ms = e0.elapsed_time(e1)
+    ms_max = fdist.max_over_ranks(ms, device if args.gpus > 1 else None)
+    value = fdist.aggregate_throughput([flops * args.steps] * world, ms_max) / 1e12
+    if fa.fa_last_device_status() != 0:
+        raise RuntimeError("device status after the timed region is not ok")
+
+    # ---------------- dominant kernel roofline
+    dom = max(prof, key=lambda k: prof[k][0])
+    dom_ms, dom_n = prof[dom]
+    per_launch_ms = dom_ms / max(dom_n, 1)
+    burst, sustained, hbm, src = peaks()
+    if dom in ("fwd", "bwd_main"):
+        alg = fwd_f if dom == "fwd" else bwd_f
+        achieved = alg / (per_launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                "frac": achieved / burst, "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)",
+                "kernel": dom, "launch_ms": per_launch_ms}
+    else:
+        alg_bytes = None
+        roof = {"bound": "hbm", "achieved": alg_bytes, "peak": hbm, "unit": "GB/s", "frac": None, "kernel": dom}
+    roof["traffic"] = traffic_for(dom, name)
+    kernel_times = {k: {"ms_per_launch": (v[0] / v[1] if v[1] else 0.0), "launches": v[1],
+                        "share": v[0] / max(sum(x[0] for x in prof.values()), 1e-12)} for k, v in prof.items()}
+    fwd_ms = prof["fwd"][0] / max(prof["fwd"][1], 1)
+    split = {"fwd_tflops": fwd_f / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
+             "fwd_frac_of_peak": (fwd_f / (fwd_ms / 1e3) / 1e12) / burst if fwd_ms else None}
+    if w["bwd"]:
+        bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post")) / max(prof["bwd_main"][1], 1)
+        split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12
+        split["bwd_frac_of_peak"] = split["bwd_tflops"] / burst
+
+    # ---------------- end to end through host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "do") if host[n] is not None}
+        outs = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True)
+                for n in (["o", "lse", "dq", "dk", "dv"] if w["bwd"] else ["o", "lse"])}
+        h2d = sum(x.numel() * x.element_size() for x in pin.values())
+        d2h = sum(x.numel() * x.element_size() for x in outs.values())
+        fdist.barrier(device)
+        torch.cuda.synchronize(device)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            for n, x in pin.items():
+                t[n].copy_(x, non_blocking=True)
+            step(w, t, stream)
+            for n, x in outs.items():
+                x.copy_(t[n], non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = fdist.max_over_ranks(a0.elapsed_time(a1), device if args.gpus > 1 else None)
+        e2e = {"value": fdist.aggregate_throughput([flops * args.e2e_steps] * world, e2e_ms) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    # ---------------- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads, secs, val = cpu_sample(host, w, kept, args.cpu_seconds)
+        cpu = {"value": val, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"{heads} of {w['B'] * w['H']} (batch, head) pairs, each: forward on all rows, "
+                         f"dQ on all rows, dK/dV on all keys; {secs:.1f} s"}
+
+    in_bytes = sum(x.numel() * x.element_size() for x in (t["q"], t["k"], t["v"]) + ((t["do"],) if w["bwd"] else ()))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+        "config": {"workload": describe(name, w), "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+                   "causal": w["causal"], "block_sparse": w["sparse"],
+                   "kept_blocks": kept, "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": ("inputs larger than L2, no flush" if in_bytes > L2_BYTES
+                          else "inputs smaller than L2 (no flush)"),
+                   "input_bytes": in_bytes},
+        "split": split,
+        "kernels": kernel_times,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": sum(v[1] for v in prof.values()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    fdist.shutdown()
+
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, args.workload)
+    else:
+        run_ours(args, w, args.workload)
+
+
+if __name__ == "__main__":
+    main()

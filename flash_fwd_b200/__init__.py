@@ -14,7 +14,7 @@ import torch
 __all__ = [
     "FaError", "load_library", "library_path", "fa_fwd", "fa_fwd_blocksparse", "fa_bwd",
     "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status",
-    "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK",
+    "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
 ]
 
 FA_BLOCK = 128
@@ -55,8 +55,10 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
     lib.fa_version.argtypes = []
+    lib.fa_profile_enable.argtypes = [i]
+    lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse,
-               lib.fa_last_device_status, lib.fa_version):
+               lib.fa_last_device_status, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -72,6 +74,21 @@ def fa_last_device_status():
 
 def fa_version():
     return load_library().fa_version()
+
+
+PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post")
+
+
+def fa_profile_enable(on=True):
+    _check(load_library().fa_profile_enable(int(bool(on))), "fa_profile_enable")
+
+
+def fa_profile_read():
+    """{kind: (milliseconds, launches)} summed since the last read."""
+    ms = (ctypes.c_float * 4)()
+    n = (ctypes.c_int * 4)()
+    _check(load_library().fa_profile_read(ms, n), "fa_profile_read")
+    return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(PROFILE_KINDS)}
 
 
 def fa_bwd_workspace_bytes(B, H, N, d):

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "fa.h"
 #include "fa_bwd.cuh"
@@ -15,6 +16,38 @@
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- profiling
+struct ProfRecord {
+    int kind;
+    cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+
+// Records events around one kernel launch when profiling is on.
+class ProfScope {
+   public:
+    ProfScope(int kind, cudaStream_t s) : kind_(kind), s_(s) {
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        if (!g_prof_on) return;
+        if (cudaEventCreate(&a_) != cudaSuccess || cudaEventCreate(&b_) != cudaSuccess) return;
+        active_ = cudaEventRecord(a_, s_) == cudaSuccess;
+    }
+    ~ProfScope() {
+        if (!active_) return;
+        cudaEventRecord(b_, s_);
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        g_prof.push_back({kind_, a_, b_});
+    }
+
+   private:
+    int kind_;
+    cudaStream_t s_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
+    bool active_ = false;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -70,6 +103,7 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     dim3 grid(BH, (p.nqb + NQ - 1) / NQ);
+    ProfScope prof(0, stream);
     kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -123,6 +157,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         constexpr int TPR = D / 8;
         const long long threads = rows * TPR;
         const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        ProfScope prof(1, stream);
         fa::bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
             static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), dvec, reinterpret_cast<float4 *>(dqacc),
             rows);
@@ -151,12 +186,16 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     dim3 grid(p.nkb * DSPLIT, BH);
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, p);
+    {
+        ProfScope prof(2, stream);
+        kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, p);
+    }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     // dQ = scale * dQacc
     {
         const long long n8 = rows * D / 8;
         const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+        ProfScope prof(3, stream);
         fa::bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dqacc),
                                                                static_cast<uint4 *>(dq), scale, n8);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -262,6 +301,36 @@ FA_API int fa_last_device_status(void) {
     if (cudaMemcpyFromSymbol(&v, fa::g_dev_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
     if (cudaMemcpyToSymbol(fa::g_dev_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
     return v;
+}
+
+FA_API int fa_profile_enable(int on) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_on = on != 0;
+    return FA_OK;
+}
+
+FA_API int fa_profile_read(float *ms, int *launches) {
+    if (!ms || !launches) return FA_ERR_INVALID_ARG;
+    std::vector<ProfRecord> recs;
+    {
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        recs.swap(g_prof);
+    }
+    for (int k = 0; k < FA_PROFILE_KINDS; ++k) {
+        ms[k] = 0.f;
+        launches[k] = 0;
+    }
+    int rc = FA_OK;
+    for (auto &r : recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            rc = FA_ERR_CUDA;
+        ms[r.kind] += t;
+        launches[r.kind] += 1;
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+    }
+    return rc;
 }
 
 FA_API int fa_version(void) { return 100; }

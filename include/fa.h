@@ -130,6 +130,20 @@ FA_API const char *fa_status_string(int status);
  */
 FA_API int fa_last_device_status(void);
 
+/*
+ * Per-kernel timing, for benchmarks.  While enabled (on != 0), every call
+ * records a pair of CUDA events on the caller's stream around each kernel it
+ * launches.  fa_profile_read() waits for those events, writes the summed
+ * milliseconds and launch counts per kernel kind, clears the record and
+ * returns FA_OK.  Kinds: 0 forward, 1 backward pre-pass (D and accumulator
+ * reset), 2 backward main kernel, 3 backward dQ conversion.  ms and launches
+ * are HOST arrays of FA_PROFILE_KINDS entries.  Events are created and
+ * destroyed by the library; no device memory is allocated.
+ */
+#define FA_PROFILE_KINDS 4
+FA_API int fa_profile_enable(int on);
+FA_API int fa_profile_read(float *ms, int *launches);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 FA_API int fa_version(void);
 
