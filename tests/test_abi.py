@@ -1,0 +1,108 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/fa.h declares, names every status, and rejects bad arguments with the
+documented status before any CUDA call (no pointer is dereferenced; the fake
+device addresses below are never touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import flash_fwd_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE = 0, 1, 2, 3, 4
+A = ctypes.c_void_p(0x10000)       # 16-byte aligned fake address
+M = ctypes.c_void_p(0x10001)       # misaligned
+NULL = ctypes.c_void_p(0)
+S = ctypes.c_void_p(0)             # stream
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_function():
+    lib = fa.load_library()
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in fa.h but not exported"
+
+
+def test_status_strings():
+    for code in range(0, 8):
+        assert isinstance(fa.fa_status_string(code), str) and fa.fa_status_string(code)
+    assert fa.fa_status_string(0) == "ok"
+    assert fa.fa_status_string(999) == "unknown status"
+
+
+def _fwd(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, scale=0.125, causal=0, dtype=1):
+    return fa.load_library().fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, S)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(d=32), UNSUPPORTED),
+    (dict(d=512), UNSUPPORTED),
+    (dict(B=0), INVALID),
+    (dict(H=-1), INVALID),
+    (dict(N=0), INVALID),
+    (dict(dtype=7), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(scale=float("inf")), INVALID),
+    (dict(q=NULL), INVALID),
+    (dict(lse=NULL), INVALID),
+    (dict(k=M), MISALIGNED),
+    (dict(o=M), MISALIGNED),
+    (dict(N=300_000_000), UNSUPPORTED),   # more query-block pairs than a grid dimension holds
+])
+def test_fwd_rejects(kw, expect):
+    assert _fwd(**kw) == expect
+
+
+def test_fwd_blocksparse_requires_mask():
+    lib = fa.load_library()
+    assert lib.fa_fwd_blocksparse(A, A, A, A, A, NULL, 1, 1, 128, 64, 0.1, 0, 1, S) == INVALID
+
+
+def test_workspace_bytes():
+    lib = fa.load_library()
+    B, H, N, d = 2, 3, 1000, 128
+    got = lib.fa_bwd_workspace_bytes(B, H, N, d)
+    d_bytes = (B * H * N * 4 + 255) // 256 * 256
+    assert got == d_bytes + B * H * N * d * 4
+    assert lib.fa_bwd_workspace_bytes(0, 1, 1, 64) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 1, 1, 96) == 0
+
+
+def _bwd(ws=A, ws_bytes=None, d=64, N=128, dq=A, mask=None):
+    lib = fa.load_library()
+    if ws_bytes is None:
+        ws_bytes = lib.fa_bwd_workspace_bytes(1, 1, N, d)
+    args = [A, A, A, A, A, A, dq, A, A, ws, ws_bytes]
+    tail = [1, 1, N, d, 0.125, 0, 1, S]
+    if mask is None:
+        return lib.fa_bwd(*args, *tail)
+    return lib.fa_bwd_blocksparse(*args, mask, *tail)
+
+
+def test_bwd_rejects():
+    lib = fa.load_library()
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    assert _bwd(ws=NULL) == WORKSPACE
+    assert _bwd(ws_bytes=need - 1) == WORKSPACE
+    assert _bwd(ws=M) == MISALIGNED
+    assert _bwd(dq=NULL) == INVALID
+    assert _bwd(dq=M) == MISALIGNED
+    assert _bwd(d=80) == UNSUPPORTED
+    assert _bwd(mask=NULL) == INVALID
+
+
+def test_profile_read_rejects_null():
+    lib = fa.load_library()
+    assert lib.fa_profile_read(None, None) == INVALID
+    assert lib.fa_version() >= 100
