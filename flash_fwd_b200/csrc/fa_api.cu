@@ -245,6 +245,31 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const v
                                      N, scale, causal, dtype, s);
 }
 
+// ---------------------------------------------------------------- fa_bwd_noalloc
+// Scratch for fa_bwd_noalloc, resident on every device that loads the library.
+// Host code must not use this name as a pointer: on the host it is only a
+// stand-in for the symbol, so the device address is looked up per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// The current device's address of g_noalloc_scratch, looked up on first use.
+int noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return FA_ERR_CUDA;
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = g_noalloc_addr[dev];
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -282,6 +307,19 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                     causal, dtype, stream);
 }
 
+FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                          const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                          int causal, int dtype, void *stream) {
+    int rc = check_common(B, H, N, d, scale, dtype);
+    if (rc != FA_OK) return rc;
+    const size_t need = fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d);
+    if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != FA_OK) return rc;
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, nullptr, B, H, N, d,
+                    scale, causal, dtype, stream);
+}
+
 FA_API const char *fa_status_string(int status) {
     switch (status) {
         case FA_OK: return "ok";
@@ -291,6 +329,7 @@ FA_API const char *fa_status_string(int status) {
         case FA_ERR_WORKSPACE: return "workspace missing or too small";
         case FA_ERR_CUDA: return "CUDA error";
         case FA_ERR_TIMEOUT: return "kernel wait timed out";
+        case FA_ERR_SCRATCH_LIMIT: return "problem needs more than the built-in scratch of fa_bwd_noalloc";
         default: return "unknown status";
     }
 }

@@ -62,7 +62,8 @@ typedef enum {
     FA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
     FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than fa_bwd_workspace_bytes() */
     FA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
-    FA_ERR_TIMEOUT = 6       /* a kernel gave up waiting (see fa_last_device_status) */
+    FA_ERR_TIMEOUT = 6,      /* a kernel gave up waiting (see fa_last_device_status) */
+    FA_ERR_SCRATCH_LIMIT = 7 /* fa_bwd_noalloc: the problem needs more than its built-in scratch */
 } fa_status;
 
 /* Side length of one block-mask block, in rows and keys. */
@@ -119,6 +120,36 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               const uint8_t *block_mask,
                               int B, int H, int N, int d, float scale, int causal, int dtype,
                               void *stream);
+
+/*
+ * Backward pass that allocates nothing and takes no workspace.
+ *
+ * The FlashAttention pages have no counterpart to this entry point; it exists
+ * for callers that cannot allocate device memory themselves: a plugin or
+ * custom-op interface that hands the library its input and output buffers but
+ * no allocator, or code that must not call cudaMalloc on its path (the call
+ * can synchronise the device, and it fails once a framework's caching
+ * allocator has reserved most of the memory).
+ *
+ * Same arguments and results as fa_bwd, minus the workspace.  The scratch the
+ * backward needs (fa_bwd_workspace_bytes(B, H, N, d) bytes: one fp32 per row
+ * and an fp32 dQ accumulator) comes from one array of
+ * FA_NOALLOC_SCRATCH_BYTES bytes that the library holds in device memory on
+ * every GPU that loads it, until the process exits.  Problems that need more
+ * are rejected with FA_ERR_SCRATCH_LIMIT before anything is launched.
+ *
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.  Every call on a device shares the one array, so
+ * calls whose kernels overlap on the GPU (different streams without ordering
+ * between them) race and give wrong results; order them on one stream.  The
+ * array keeps the last call's contents; each call clears what it needs zeroed.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                          const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                          int B, int H, int N, int d, float scale, int causal, int dtype,
+                          void *stream);
 
 /* A static, human-readable name for a status code. */
 FA_API const char *fa_status_string(int status);
