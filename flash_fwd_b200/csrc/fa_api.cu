@@ -146,21 +146,25 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
 }
 
 
-template <int D, int BM, int DSPLIT, int NS, bool DQT, bool BF16>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16>
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
-               void *dq, void *dk, void *dv, float *dvec, float *dqacc, const uint8_t *mask, int BH, int N,
-               float scale, int causal, int dtype, cudaStream_t stream) {
-    using C = fa::BwdCfg<D, BM, DSPLIT, NS, DQT>;
+               void *dq, void *dk, void *dv, void *workspace, const uint8_t *mask, int BH, int N, float scale,
+               int causal, int dtype, cudaStream_t stream) {
+    using C = fa::BwdCfg<D, BM, DSPLIT, NS, NPB, DQT>;
     const long long rows = static_cast<long long>(BH) * N;
-    // D = rowsum(dO o O) and dQacc = 0
+    const int Npad = fa::bwd_npad(N);
+    float *lse2 = static_cast<float *>(workspace);
+    float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
+    float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
+    // lse2 = LSE * log2(e), D = rowsum(dO o O) (padded rows: +inf, 0) and dQacc = 0
     {
         constexpr int TPR = D / 8;
-        const long long threads = rows * TPR;
+        const long long threads = static_cast<long long>(BH) * Npad * TPR;
         const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
         ProfScope prof(1, stream);
         fa::bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
-            static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), dvec, reinterpret_cast<float4 *>(dqacc),
-            rows);
+            static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), lse, lse2, dvec,
+            reinterpret_cast<float4 *>(dqacc), N, Npad, BH);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     CUtensorMap mk, mv, mq, mdo;
@@ -170,19 +174,20 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     if ((rc = make_map(&mq, q, D, N, BH, dtype, BM)) != FA_OK) return rc;
     if ((rc = make_map(&mdo, dout, D, N, BH, dtype, BM)) != FA_OK) return rc;
     fa::BwdParams p;
-    p.lse = lse;
+    p.lse2 = lse2;
     p.dvec = dvec;
     p.dqacc = dqacc;
     p.dk = dk;
     p.dv = dv;
     p.mask = mask;
     p.N = N;
+    p.Npad = Npad;
     p.nkb = (N + 127) / 128;
     p.nqt = (N + BM - 1) / BM;
     p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
-    auto kern = fa::bwd_kernel<D, BM, DSPLIT, NS, DQT, BF16>;
+    auto kern = fa::bwd_kernel<D, BM, DSPLIT, NS, NPB, DQT, BF16>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     dim3 grid(p.nkb * DSPLIT, BH);
@@ -205,17 +210,17 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 
 template <bool BF16>
 int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *o, const void *dout,
-                 const float *lse, void *dq, void *dk, void *dv, float *dvec, float *dqacc, const uint8_t *mask,
+                 const float *lse, void *dq, void *dk, void *dv, void *ws, const uint8_t *mask,
                  int BH, int N, float scale, int causal, int dtype, cudaStream_t s) {
     switch (d) {
         case 64:
-            return launch_bwd<64, 128, 1, 3, false, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+            return launch_bwd<64, 128, 1, 4, 1, false, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
                                                           N, scale, causal, dtype, s);
         case 128:
-            return launch_bwd<128, 64, 1, 3, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+            return launch_bwd<128, 64, 1, 3, 2, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
                                                          N, scale, causal, dtype, s);
         case 256:
-            return launch_bwd<256, 64, 2, 1, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, BH,
+            return launch_bwd<256, 64, 2, 1, 2, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
                                                          N, scale, causal, dtype, s);
         default: return FA_ERR_UNSUPPORTED;
     }
@@ -234,14 +239,11 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const v
     const size_t need = fa::bwd_workspace_bytes(BH, N, d);
     if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-    float *dvec = static_cast<float *>(workspace);
-    float *dqacc = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                             ((static_cast<size_t>(BH) * N * 4 + 255) & ~static_cast<size_t>(255)));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return dtype == FA_BF16
-               ? dispatch_bwd<true>(d, q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, static_cast<int>(BH), N,
+               ? dispatch_bwd<true>(d, q, k, v, o, dout, lse, dq, dk, dv, workspace, mask, static_cast<int>(BH), N,
                                     scale, causal, dtype, s)
-               : dispatch_bwd<false>(d, q, k, v, o, dout, lse, dq, dk, dv, dvec, dqacc, mask, static_cast<int>(BH),
+               : dispatch_bwd<false>(d, q, k, v, o, dout, lse, dq, dk, dv, workspace, mask, static_cast<int>(BH),
                                      N, scale, causal, dtype, s);
 }
 

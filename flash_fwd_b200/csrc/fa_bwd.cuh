@@ -36,13 +36,14 @@
 namespace fa {
 
 struct BwdParams {
-    const float *lse;     // [BH][N] natural-log LSE from the forward
-    const float *dvec;    // [BH][N] D = rowsum(dO o O)
+    const float *lse2;    // [BH][Npad] LSE * log2(e) (+inf for rows past N or with no visible key)
+    const float *dvec;    // [BH][Npad] D = rowsum(dO o O) (0 for rows past N)
     float *dqacc;         // [BH][N][D] fp32, zeroed by bwd_pre
     void *dk;             // [BH][N][D] 16-bit
     void *dv;             // [BH][N][D] 16-bit
     const uint8_t *mask;  // [nkb][nkb] block mask (kSparse)
     int N;
+    int Npad;             // N rounded up to 128: row pitch of lse2 and dvec
     int nkb;              // key blocks (and mask blocks) of 128
     int nqt;              // query tiles of BM rows
     int mode;
@@ -55,14 +56,19 @@ struct BwdParams {
 // ---------------------------------------------------------------------------
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint4 *__restrict__ o, const uint4 *__restrict__ dout,
-                                                      float *__restrict__ dvec, float4 *__restrict__ dqacc,
-                                                      long long rows) {
+                                                      const float *__restrict__ lse, float *__restrict__ lse2,
+                                                      float *__restrict__ dvec, float4 *__restrict__ dqacc, int N,
+                                                      int Npad, long long BH) {
     constexpr int TPR = D / 8;   // threads per row, 8 elements (16 bytes) each
     const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const long long row = tid / TPR;
+    const long long prow = tid / TPR;                 // padded row index bh * Npad + n
     const int part = static_cast<int>(tid % TPR);
+    const long long bh = prow / Npad;
+    const int n = static_cast<int>(prow % Npad);
+    const bool valid = bh < BH && n < N;
+    const long long row = bh * N + n;
     float acc = 0.f;
-    if (row < rows) {
+    if (valid) {
         const uint4 a = o[row * TPR + part];
         const uint4 b = dout[row * TPR + part];
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -78,7 +84,15 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint4 *__restrict__ 
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (row < rows && part == 0) dvec[row] = acc;
+    if (bh < BH && part == 0) {
+        float l2 = INFINITY;      // P = 2^(s - inf) = 0 for rows past N or with no visible key
+        if (valid) {
+            const float L = lse[row];
+            if (L != -INFINITY) l2 = L * 1.4426950408889634f;
+        }
+        lse2[prow] = l2;
+        dvec[prow] = valid ? acc : 0.f;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -123,7 +137,7 @@ struct QIter {
     }
 };
 
-template <int D, int BM, int DSPLIT, int NS, bool DQT>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT>
 struct BwdCfg {
     static constexpr int DH = D / DSPLIT;                 // output columns per CTA
     static constexpr int kKVTile = 128 * D * 2;           // K_j or V_j
@@ -135,9 +149,8 @@ struct BwdCfg {
     static constexpr int kVOff = kKOff + kKVTile;
     static constexpr int kQOff = kVOff + kKVTile;
     static constexpr int kdOOff = kQOff + NS * kQTile;
-    static constexpr int kPOff = kdOOff + NS * kQTile;
-    static constexpr int kdSOff = kPOff + kPTile;
-    static constexpr int kStatOff = kdSOff + kPTile;      // per stage: lse*log2e [BM], D [BM]
+    static constexpr int kdSOff = kdOOff + NS * kQTile;   // NPB buffers of dS^T
+    static constexpr int kStatOff = kdSOff + NPB * kPTile;   // per stage: lse*log2e [BM], D [BM]
     static constexpr int kBarOff = kStatOff + NS * BM * 8;
     static constexpr int kBarKV = 0;
     static constexpr int kBarQFull = 1;
@@ -145,8 +158,8 @@ struct BwdCfg {
     static constexpr int kBarSdpFull = kBarQEmpty + NS;
     static constexpr int kBarSdpEmpty = kBarSdpFull + 1;
     static constexpr int kBarDsFull = kBarSdpEmpty + 1;
-    static constexpr int kBarPdsEmpty = kBarDsFull + 1;
-    static constexpr int kBarDqFull = kBarPdsEmpty + 1;
+    static constexpr int kBarPdsEmpty = kBarDsFull + 1;   // NPB barriers, one per P/dS buffer
+    static constexpr int kBarDqFull = kBarPdsEmpty + NPB;
     static constexpr int kBarDqEmpty = kBarDqFull + 1;
     static constexpr int kBarMmaDone = kBarDqEmpty + 1;
     static constexpr int kNumBars = kBarMmaDone + 1;
@@ -159,17 +172,21 @@ struct BwdCfg {
     static constexpr int kColDK = 256 + DH;
     static constexpr int kColDQ = DQT ? 64 : 256 + 2 * DH;
     static constexpr int kDqCols = DQT ? BM : DH;         // fp32 columns per drain thread
+    static constexpr int kColPT = DQT ? 192 : 448;        // NPB buffers of 16-bit P^T (BM / 2 columns each)
+    static constexpr int kStatBytes = BM * 4;
+    static_assert(kColPT + NPB * BM / 2 <= (DQT ? 256 : 512), "P^T columns");
     static_assert(DQT ? (BM == 64 && DH == 128) : (BM == 128 && DH == 64), "tile shape");
     static_assert(kColDQ + kDqCols <= 512 && kColDK + DH <= 512, "TMEM columns");
+    static_assert(NPB == 1 || NPB == 2, "P/dS buffers");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BM, int DSPLIT, int NS, bool DQT, bool BF16>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16>
 __global__ void __launch_bounds__(320, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
                const BwdParams p) {
-    using C = BwdCfg<D, BM, DSPLIT, NS, DQT>;
+    using C = BwdCfg<D, BM, DSPLIT, NS, NPB, DQT>;
     constexpr int DH = C::DH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(bar(C::kBarSdpFull), 1);
         mbar_init(bar(C::kBarSdpEmpty), 128);
         mbar_init(bar(C::kBarDsFull), 128);
-        mbar_init(bar(C::kBarPdsEmpty), 1);
+        for (int b = 0; b < NPB; ++b) mbar_init(bar(C::kBarPdsEmpty + b), 1);
         mbar_init(bar(C::kBarDqFull), 1);
         mbar_init(bar(C::kBarDqEmpty), 128);
         mbar_init(bar(C::kBarMmaDone), 1);
@@ -235,27 +252,19 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t ph = (cnt / NS) & 1;
             ok = wait_bar(bar(C::kBarQEmpty + s), ph ^ 1u, abort_flag);
             if (!ok) break;
-            float *st = reinterpret_cast<float *>(smem + C::kStatOff + s * BM * 8);
-            for (int k = lane; k < BM; k += 32) {
-                const int q = i * BM + k;
-                float l2 = INFINITY, dd = 0.f;     // rows past N (or with no visible key) give P = 0
-                if (q < p.N) {
-                    const float L = p.lse[static_cast<size_t>(bh) * p.N + q];
-                    if (L != -INFINITY) l2 = L * 1.4426950408889634f;
-                    dd = p.dvec[static_cast<size_t>(bh) * p.N + q];
-                }
-                st[k] = l2;
-                st[BM + k] = dd;
-            }
-            __syncwarp();
+            // Q_i, dO_i (TMA tiles) and the padded per-row statistics (bulk
+            // copies, prepared by bwd_pre) land on one transaction barrier
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarQFull + s), 2 * C::kQTile);
+                const uint32_t qb = bar(C::kBarQFull + s);
+                mbar_arrive_expect_tx(qb, 2 * C::kQTile + 2 * C::kStatBytes);
                 for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, bar(C::kBarQFull + s),
-                                c * 64, i * BM, bh);
-                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo,
-                                bar(C::kBarQFull + s), c * 64, i * BM, bh);
+                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, qb, c * 64, i * BM, bh);
+                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo, qb, c * 64, i * BM, bh);
                 }
+                const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
+                bulk_load(sbase + C::kStatOff + s * 2 * C::kStatBytes, p.lse2 + srow, C::kStatBytes, qb);
+                bulk_load(sbase + C::kStatOff + s * 2 * C::kStatBytes + C::kStatBytes, p.dvec + srow,
+                          C::kStatBytes, qb);
             }
             __syncwarp();
             ++cnt;
@@ -268,53 +277,53 @@ __global__ void __launch_bounds__(320, 1)
         constexpr uint32_t kIdKV = instr_desc_f16(128, DH, BF16, false, true);
         constexpr uint32_t kIdQ = DQT ? instr_desc_f16(128, BM, BF16, true, true)
                                       : instr_desc_f16(128, DH, BF16, true, true);
-        const uint32_t sK = sbase + C::kKOff, sV = sbase + C::kVOff;
-        const uint32_t sP = sbase + C::kPOff, sdS = sbase + C::kdSOff;
+        // descriptors built once; each instruction only offsets the start address
+        const SmemDesc dK_kmaj = make_desc(sbase + C::kKOff, 16, 1024);
+        const SmemDesc dV_kmaj = make_desc(sbase + C::kVOff, 16, 1024);
+        const SmemDesc dQ_kmaj = make_desc(sbase + C::kQOff, 16, 1024);
+        const SmemDesc ddO_kmaj = make_desc(sbase + C::kdOOff, 16, 1024);
+        const SmemDesc dQ_mn = make_desc(sbase + C::kQOff + h * (DH / 64) * C::kQChunk, C::kQChunk, 1024);
+        const SmemDesc ddO_mn = make_desc(sbase + C::kdOOff + h * (DH / 64) * C::kQChunk, C::kQChunk, 1024);
+        const SmemDesc ddS_kmaj = make_desc(sbase + C::kdSOff, 16, 1024);
+        const SmemDesc ddS_mn = make_desc(sbase + C::kdSOff, 128 * 128, 1024);
+        const SmemDesc dK_mn = make_desc(sbase + C::kKOff + h * (DH / 64) * C::kKVChunk, C::kKVChunk, 1024);
         auto issue_sdp = [&](int s) {
-            const uint32_t sQ = sbase + C::kQOff + s * C::kQTile, sdO = sbase + C::kdOOff + s * C::kQTile;
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
-                const uint32_t oq = (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColS, smem_desc_sw128(sK + okv, 16, 1024), smem_desc_sw128(sQ + oq, 16, 1024),
-                       kIdS, k > 0 ? 1u : 0u);
+                const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
+                mma_ss(tmem + C::kColS, dK_kmaj.at(okv), dQ_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
-                const uint32_t oq = (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColDP, smem_desc_sw128(sV + okv, 16, 1024),
-                       smem_desc_sw128(sdO + oq, 16, 1024), kIdS, k > 0 ? 1u : 0u);
+                const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
+                mma_ss(tmem + C::kColDP, dV_kmaj.at(okv), ddO_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
             }
         };
-        auto issue_dvdk = [&](int s, bool acc) {
-            const uint32_t sQ = sbase + C::kQOff + s * C::kQTile, sdO = sbase + C::kdOOff + s * C::kQTile;
-            const uint32_t half = h * (DH / 64) * C::kQChunk;
+        auto issue_dvdk = [&](int s, int pb, bool acc) {
+#pragma unroll
+            for (int k = 0; k < BM / 16; ++k)   // dV += P^T dO_i, P^T read from TMEM
+                mma_ts(tmem + C::kColDV, tmem + C::kColPT + pb * (BM / 2) + 8 * k,
+                       ddO_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < BM / 16; ++k) {
-                const uint32_t oa = (k >> 2) * (128 * 128) + (k & 3) * 32;
-                mma_ss(tmem + C::kColDV, smem_desc_sw128(sP + oa, 16, 1024),
-                       smem_desc_sw128(sdO + half + k * 2048, C::kQChunk, 1024), kIdKV, (acc || k > 0) ? 1u : 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < BM / 16; ++k) {
-                const uint32_t oa = (k >> 2) * (128 * 128) + (k & 3) * 32;
-                mma_ss(tmem + C::kColDK, smem_desc_sw128(sdS + oa, 16, 1024),
-                       smem_desc_sw128(sQ + half + k * 2048, C::kQChunk, 1024), kIdKV, (acc || k > 0) ? 1u : 0u);
+                const uint32_t oa = pb * C::kPTile + (k >> 2) * (128 * 128) + (k & 3) * 32;
+                mma_ss(tmem + C::kColDK, ddS_kmaj.at(oa), dQ_mn.at(s * C::kQTile + k * 2048), kIdKV,
+                       (acc || k > 0) ? 1u : 0u);
             }
         };
-        auto issue_dq = [&]() {
+        auto issue_dq = [&](int pb) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 if constexpr (DQT) {
                     // dQ^T (DH x BM) = K_j^T (DH x 128 keys) * dS^T (128 keys x BM)
-                    mma_ss(tmem + C::kColDQ,
-                           smem_desc_sw128(sK + h * (DH / 64) * C::kKVChunk + k * 2048, C::kKVChunk, 1024),
-                           smem_desc_sw128(sdS + k * 2048, 128 * 128, 1024), kIdQ, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColDQ, dK_mn.at(k * 2048), ddS_mn.at(pb * C::kPTile + k * 2048), kIdQ,
+                           k > 0 ? 1u : 0u);
                 } else {
                     // dQ (BM x DH) = dS (BM x 128 keys) * K_j (128 keys x DH)
-                    mma_ss(tmem + C::kColDQ, smem_desc_sw128(sdS + k * 2048, 128 * 128, 1024),
-                           smem_desc_sw128(sK + k * 2048, C::kKVChunk, 1024), kIdQ, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColDQ, ddS_mn.at(pb * C::kPTile + k * 2048), dK_mn.at(k * 2048), kIdQ,
+                           k > 0 ? 1u : 0u);
                 }
             }
         };
@@ -350,6 +359,7 @@ __global__ void __launch_bounds__(320, 1)
         };
         while (ok && have) {
             const int s = cnt % NS;
+            const int pb = cnt % NPB;
             const bool have_n = it.next(p, j, in);
             // with two or more stages the next tile is already resident: overlap
             // its S^T, dP^T with this tile's softmax-grad work.  With one stage
@@ -361,15 +371,15 @@ __global__ void __launch_bounds__(320, 1)
             ok = wait_bar(bar(C::kBarDsFull), cnt & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            if (lane == 0) issue_dvdk(s, cnt > 0);
+            if (lane == 0) issue_dvdk(s, pb, cnt > 0);
             __syncwarp();
             ok = wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                issue_dq();
+                issue_dq(pb);
                 mma_commit(bar(C::kBarDqFull));
-                mma_commit(bar(C::kBarPdsEmpty));
+                mma_commit(bar(C::kBarPdsEmpty + pb));
                 mma_commit(bar(C::kBarQEmpty + s));
             }
             __syncwarp();
@@ -390,18 +400,19 @@ __global__ void __launch_bounds__(320, 1)
         const int r = warp * 32 + lane;     // key row within the block
         const int key = j * 128 + r;
         const float c = p.scale_log2;
-        uint8_t *sP = smem + C::kPOff;
-        uint8_t *sdS = smem + C::kdSOff;
         QIter<BM> it;
         int i;
         while (it.next(p, j, i)) {
             const int s = cnt % NS;
+            const int pb = cnt % NPB;
+            uint8_t *sdS = smem + C::kdSOff + pb * C::kPTile;
+            const uint32_t tP = tmem + lane_off + C::kColPT + pb * (BM / 2);
             ok = wait_bar(bar(C::kBarSdpFull), cnt & 1, abort_flag) &&
                  wait_bar(bar(C::kBarQFull + s), (cnt / NS) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const float *lse2 = reinterpret_cast<const float *>(smem + C::kStatOff + s * BM * 8);
-            const float *dd = lse2 + BM;
+            const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
+            const float4 *dd4 = lse4 + BM / 4;
             const bool need_causal = (p.mode & kCausal) && (i * BM < j * 128 + 127);
 #pragma unroll 1
             for (int ch = 0; ch < BM / 32; ++ch) {
@@ -415,37 +426,46 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    float pp[2], ds[2];
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    const float4 l4 = lse4[ch * 8 + k4];
+                    const float4 d4 = dd4[ch * 8 + k4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pp[4], ds[4];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = 32 * ch + 2 * k + e;
-                        float pv = ex2(fmaf(__uint_as_float(sr[2 * k + e]), c, -lse2[col]));
-                        if (need_causal && key > i * BM + col) pv = 0.f;
+                    for (int e = 0; e < 4; ++e) {
+                        const int kk = 4 * k4 + e;
+                        float pv = ex2(fmaf(__uint_as_float(sr[kk]), c, -lv[e]));
+                        if (need_causal && key > i * BM + 32 * ch + kk) pv = 0.f;
                         pp[e] = pv;
-                        ds[e] = pv * (__uint_as_float(pr[2 * k + e]) - dd[col]);
+                        ds[e] = pv * (__uint_as_float(pr[kk]) - dv[e]);
                     }
-                    pk[k] = pack2<BF16>(pp[0], pp[1]);
-                    dk[k] = pack2<BF16>(ds[0], ds[1]);
+                    pk[2 * k4] = pack2<BF16>(pp[0], pp[1]);
+                    pk[2 * k4 + 1] = pack2<BF16>(pp[2], pp[3]);
+                    dk[2 * k4] = pack2<BF16>(ds[0], ds[1]);
+                    dk[2 * k4 + 1] = pack2<BF16>(ds[2], ds[3]);
                 }
-                if (ch == 0 && cnt > 0) {
-                    // the previous tile's dV/dK/dQ products must be done reading P^T, dS^T
-                    if (!wait_bar(bar(C::kBarPdsEmpty), (cnt - 1) & 1, abort_flag)) {
+                if (ch == 0 && cnt >= NPB) {
+                    // the products that read this P/dS buffer NPB tiles ago must be done
+                    if (!wait_bar(bar(C::kBarPdsEmpty + pb), ((cnt / NPB) - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                 }
-                // row r of a K-major [BM/64][128][64] 128B-swizzled tile
+                // P^T row r -> TMEM (A operand of dV); dS^T row r -> a K-major
+                // [BM/64][128][64] 128B-swizzled shared tile (dK and dQ operand)
+                tmem_st16(tP + 16 * ch, pk);
                 const int chunk = (32 * ch) / 64;
                 const int u0 = ((32 * ch) % 64) / 8;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int off = chunk * (128 * 128) + r * 128 + (((u0 + u) ^ (r & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(sP + off) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                     *reinterpret_cast<uint4 *>(sdS + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
                 }
             }
             if (!ok) break;
+            tmem_st_wait();
+            tc_fence_before();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(bar(C::kBarDsFull));
             ++cnt;
@@ -534,9 +554,11 @@ __global__ void __launch_bounds__(320, 1)
     }
 }
 
+// Workspace: lse2 [BH][Npad] and D [BH][Npad] fp32 (Npad = N rounded up to
+// 128), then the fp32 dQ accumulator [BH][N][d].
+inline int bwd_npad(int N) { return (N + 127) / 128 * 128; }
 inline size_t bwd_workspace_bytes(long long BH, int N, int d) {
-    const size_t dbytes = (static_cast<size_t>(BH) * N * 4 + 255) & ~static_cast<size_t>(255);
-    return dbytes + static_cast<size_t>(BH) * N * d * 4;
+    return 2 * static_cast<size_t>(BH) * bwd_npad(N) * 4 + static_cast<size_t>(BH) * N * d * 4;
 }
 
 }  // namespace fa

@@ -59,6 +59,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// Raises the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -108,6 +113,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Contiguous bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
         : "memory");
 }
 
@@ -225,6 +238,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     desc |= 1ull << 46;   // descriptor version for sm_100
     desc |= 2ull << 61;   // 128-byte swizzle
     return desc;
+}
+
+// The descriptor split in halves: `hi` (strides, version, swizzle) is fixed
+// for an operand tile, `lo` holds the start address (bits 0-13) and LBO.
+// Stepping through a tile only adds (byte offset >> 4) to `lo`, which never
+// carries out of the 14-bit address field inside shared memory.
+struct SmemDesc {
+    uint32_t lo, hi;
+    __device__ __forceinline__ uint64_t at(uint32_t byte_off) const {
+        return (static_cast<uint64_t>(hi) << 32) | (lo + (byte_off >> 4));
+    }
+};
+__device__ __forceinline__ SmemDesc make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    const uint64_t d = smem_desc_sw128(saddr, lbo, sbo);
+    return SmemDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
 }
 
 // Instruction descriptor for kind::f16 with fp32 accumulation.

@@ -230,25 +230,26 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t kIdescS = instr_desc_f16(128, 128, BF16, false, false);
         constexpr uint32_t kIdescO = instr_desc_f16(128, D, BF16, false, true);
+        // descriptors built once; each instruction only offsets the start address
+        const SmemDesc dQ = make_desc(sbase + C::kQOff, 16, 1024);
+        const SmemDesc dK = make_desc(sbase + C::kKOff, 16, 1024);
+        const SmemDesc dV = make_desc(sbase + C::kVOff, C::kChunkBytes, 1024);
         auto issue_s = [&](int t, int s) {
-            const uint32_t a0 = sbase + C::kQOff + t * C::kTileBytes;
-            const uint32_t b0 = sbase + C::kKOff + s * C::kTileBytes;
             const uint32_t d_tmem = tmem + 128u * t;
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t koff = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
-                mma_ss(d_tmem, smem_desc_sw128(a0 + koff, 16, 1024),
-                       smem_desc_sw128(b0 + koff, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+                mma_ss(d_tmem, dQ.at(t * C::kTileBytes + koff), dK.at(s * C::kTileBytes + koff), kIdescS,
+                       k > 0 ? 1u : 0u);
             }
         };
         auto issue_pv = [&](int t, int s, bool acc) {
-            const uint32_t b0 = sbase + C::kVOff + s * C::kTileBytes;
             const uint32_t d_tmem = tmem + C::kOCol + D * t;
             const uint32_t a_tmem = tmem + 128u * t;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                mma_ts(d_tmem, a_tmem + 8u * k, smem_desc_sw128(b0 + k * 2048, C::kChunkBytes, 1024),
-                       kIdescO, (acc || k > 0) ? 1u : 0u);
+                mma_ts(d_tmem, a_tmem + 8u * k, dV.at(s * C::kTileBytes + k * 2048), kIdescO,
+                       (acc || k > 0) ? 1u : 0u);
         };
 
         KvIter<NQ> it;

@@ -93,8 +93,10 @@ FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void 
                               void *stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: an fp32 D = rowsum(dO * O) per row
- * and an fp32 dQ accumulator [B][H][N][d].  Returns 0 for invalid sizes.
+ * Bytes of device workspace fa_bwd needs: two fp32 per-row statistics
+ * (LSE * log2 e and D = rowsum(dO * O)), each [B][H][Npad] with N padded up
+ * to a multiple of FA_BLOCK, then an fp32 dQ accumulator [B][H][N][d].
+ * Returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
