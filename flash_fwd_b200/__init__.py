@@ -13,7 +13,7 @@ import torch
 
 __all__ = [
     "FaError", "load_library", "library_path", "fa_fwd", "fa_fwd_blocksparse", "fa_bwd",
-    "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status",
+    "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status", "fa_last_timeout_site",
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
 ]
 
@@ -55,10 +55,11 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
     lib.fa_version.argtypes = []
+    lib.fa_last_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse,
-               lib.fa_last_device_status, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
+               lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -70,6 +71,15 @@ def fa_status_string(status):
 
 def fa_last_device_status():
     return load_library().fa_last_device_status()
+
+
+def fa_last_timeout_site():
+    """(block x, block y, warp, mbarrier shared address, parity) of the first wait that gave up."""
+    site = (ctypes.c_int * 5)()
+    rc = load_library().fa_last_timeout_site(site)
+    if rc != 0:
+        raise FaError(rc, "fa_last_timeout_site")
+    return tuple(site)
 
 
 def fa_version():

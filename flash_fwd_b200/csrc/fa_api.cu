@@ -344,6 +344,13 @@ FA_API int fa_last_device_status(void) {
     return v;
 }
 
+FA_API int fa_last_timeout_site(int *site) {
+    if (!site) return FA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(site, fa::g_dev_site, 5 * sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+}
+
 FA_API int fa_profile_enable(int on) {
     std::lock_guard<std::mutex> g(g_prof_mu);
     g_prof_on = on != 0;

@@ -22,6 +22,10 @@ namespace fa {
 // Device error word (one per device that loads the library; every kernel of
 // the library is compiled into the one translation unit fa_api.cu).
 static __device__ int g_dev_status = 0;
+// Where the first wait that gave up was: block x, block y, warp, shared
+// address of its mbarrier, parity waited for.  Written only by the thread
+// whose timeout set g_dev_status.
+static __device__ int g_dev_site[5];
 
 constexpr int kErrTimeout = 6;           // matches FA_ERR_TIMEOUT
 constexpr unsigned long long kTimeoutNs = 3000000000ull;   // 3 s per wait
@@ -91,7 +95,13 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
                 if (*abort_flag) break;
                 if (globaltimer() - t0 > kTimeoutNs) {
                     *abort_flag = 1;
-                    atomicCAS(&g_dev_status, 0, kErrTimeout);
+                    if (atomicCAS(&g_dev_status, 0, kErrTimeout) == 0) {
+                        g_dev_site[0] = static_cast<int>(blockIdx.x);
+                        g_dev_site[1] = static_cast<int>(blockIdx.y);
+                        g_dev_site[2] = static_cast<int>(threadIdx.x >> 5);
+                        g_dev_site[3] = static_cast<int>(bar);
+                        g_dev_site[4] = static_cast<int>(parity);
+                    }
                     break;
                 }
             }

@@ -164,6 +164,15 @@ FA_API const char *fa_status_string(int status);
 FA_API int fa_last_device_status(void);
 
 /*
+ * Where the first wait that gave up (FA_ERR_TIMEOUT) was, for diagnosis:
+ * site[0..4] = block x, block y, warp, shared-memory address of the
+ * mbarrier, phase parity waited for.  site is a HOST array of 5 ints.  The
+ * record is kept until a later timeout overwrites it (it is not cleared by
+ * fa_last_device_status).  Synchronises the current device.
+ */
+FA_API int fa_last_timeout_site(int *site);
+
+/*
  * Per-kernel timing, for benchmarks.  While enabled (on != 0), every call
  * records a pair of CUDA events on the caller's stream around each kernel it
  * launches.  fa_profile_read() waits for those events, writes the summed
