@@ -11,6 +11,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_split.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -146,29 +147,45 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
 }
 
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16>
-int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
-               void *dq, void *dk, void *dv, void *workspace, const uint8_t *mask, int BH, int N, float scale,
-               int causal, int dtype, cudaStream_t stream) {
-    using C = fa::BwdCfg<D, BM, DSPLIT, NS, NPB, DQT>;
-    const long long rows = static_cast<long long>(BH) * N;
+// D = rowsum(dO o O), LSE * log2(e) (padded rows: +inf) and dQacc = 0.
+template <int D, bool BF16>
+int launch_bwd_pre(const void *o, const void *dout, const float *lse, float *lse2, float *dvec, float *dqacc,
+                   int BH, int N, int Npad, cudaStream_t stream) {
+    constexpr int TPR = D / 8;
+    const long long threads = static_cast<long long>(BH) * Npad * TPR;
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    ProfScope prof(1, stream);
+    fa::bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
+        static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), lse, lse2, dvec,
+        reinterpret_cast<float4 *>(dqacc), N, Npad, BH);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// dQ = scale * dQacc in the 16-bit type.
+template <bool BF16>
+int launch_bwd_post(const float *dqacc, void *dq, long long elems, float scale, cudaStream_t stream) {
+    const long long n8 = elems / 8;
+    const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+    ProfScope prof(3, stream);
+    fa::bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dqacc),
+                                                           static_cast<uint4 *>(dq), scale, n8);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Three launches: pre-pass, main kernel (Kernel: a bwd_kernel or bwd_split_kernel
+// instantiation, BM query rows per tile, grid from MakeGrid), post-pass.
+template <int D, int BM, bool BF16, typename Kernel, typename MakeGrid>
+int launch_bwd(Kernel kern, int smem_bytes, int threads, MakeGrid make_grid, const void *q, const void *k,
+               const void *v, const void *o, const void *dout, const float *lse, void *dq, void *dk, void *dv,
+               void *workspace, const uint8_t *mask, int BH, int N, float scale, int causal, int dtype,
+               cudaStream_t stream) {
     const int Npad = fa::bwd_npad(N);
     float *lse2 = static_cast<float *>(workspace);
     float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
     float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
-    // lse2 = LSE * log2(e), D = rowsum(dO o O) (padded rows: +inf, 0) and dQacc = 0
-    {
-        constexpr int TPR = D / 8;
-        const long long threads = static_cast<long long>(BH) * Npad * TPR;
-        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-        ProfScope prof(1, stream);
-        fa::bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
-            static_cast<const uint4 *>(o), static_cast<const uint4 *>(dout), lse, lse2, dvec,
-            reinterpret_cast<float4 *>(dqacc), N, Npad, BH);
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    }
+    int rc = launch_bwd_pre<D, BF16>(o, dout, lse, lse2, dvec, dqacc, BH, N, Npad, stream);
+    if (rc != FA_OK) return rc;
     CUtensorMap mk, mv, mq, mdo;
-    int rc;
     if ((rc = make_map(&mk, k, D, N, BH, dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mv, v, D, N, BH, dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mq, q, D, N, BH, dtype, BM)) != FA_OK) return rc;
@@ -187,41 +204,43 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
-    auto kern = fa::bwd_kernel<D, BM, DSPLIT, NS, NPB, DQT, BF16>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
         return FA_ERR_CUDA;
-    dim3 grid(p.nkb * DSPLIT, BH);
     {
         ProfScope prof(2, stream);
-        kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, p);
+        kern<<<make_grid(p.nkb, BH), threads, smem_bytes, stream>>>(mk, mv, mq, mdo, p);
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    // dQ = scale * dQacc
-    {
-        const long long n8 = rows * D / 8;
-        const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
-        ProfScope prof(3, stream);
-        fa::bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dqacc),
-                                                               static_cast<uint4 *>(dq), scale, n8);
-        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    }
-    return FA_OK;
+    return launch_bwd_post<BF16>(dqacc, dq, static_cast<long long>(BH) * N * D, scale, stream);
 }
 
 template <bool BF16>
 int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, void *ws, const uint8_t *mask,
                  int BH, int N, float scale, int causal, int dtype, cudaStream_t s) {
+    // d <= 128: grid (BH, key blocks), so that the heaviest causal key blocks
+    // (j = 0) are scheduled first.  d = 256: two CTAs per key block.
+    auto grid_bh_j = [](int nkb, int bh) { return dim3(bh, nkb); };
+    auto grid_split = [](int nkb, int bh) { return dim3(nkb * 2, bh); };
     switch (d) {
-        case 64:
-            return launch_bwd<64, 128, 1, 4, 1, false, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
-                                                          N, scale, causal, dtype, s);
-        case 128:
-            return launch_bwd<128, 64, 1, 3, 2, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
-                                                         N, scale, causal, dtype, s);
-        case 256:
-            return launch_bwd<256, 64, 2, 1, 2, true, BF16>(q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH,
-                                                         N, scale, causal, dtype, s);
+        case 64: {
+            using C = fa::BwdCfg<64, 3>;
+            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16>, C::kSmemBytes, C::kThreads, grid_bh_j,
+                                             q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH, N, scale, causal,
+                                             dtype, s);
+        }
+        case 128: {
+            using C = fa::BwdCfg<128, 2>;
+            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16>, C::kSmemBytes, C::kThreads, grid_bh_j,
+                                              q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH, N, scale, causal,
+                                              dtype, s);
+        }
+        case 256: {
+            using C = fa::BwdSplitCfg<256, 64, 2, 1, 2, true>;
+            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16>, C::kSmemBytes,
+                                             C::kThreads, grid_split, q, k, v, o, dout, lse, dq, dk, dv, ws, mask,
+                                             BH, N, scale, causal, dtype, s);
+        }
         default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -236,6 +255,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const v
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
     const long long BH = static_cast<long long>(B) * H;
+    if ((N + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;   // key blocks index grid.y
     const size_t need = fa::bwd_workspace_bytes(BH, N, d);
     if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FA_ERR_MISALIGNED;

@@ -137,66 +137,99 @@ struct QIter {
     }
 };
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT>
+// ---------------------------------------------------------------------------
+// bwd_kernel (d = 64, 128): one CTA per 128-key block j, query tiles of 128.
+//
+// Every product is a full-rate tcgen05 shape (M = 128 or d, N = 128):
+//   S^T  = K_j Q_i^T        SS    -> TMEM [0, 128)        (lane = key)
+//   dP^T = V_j dO_i^T       SS    -> TMEM [128, 256)
+//   dV  += P^T dO_i         TS    P^T (16-bit) written by the softmax-grad
+//                                 warps over the S^T columns they have read
+//   dK  += dS^T Q_i         SS    dS^T (16-bit) in shared memory
+//   dQ_i^T = K_j^T dS^T     SS    -> TMEM [128, 256) once dP^T has been read
+//                                 (lane = d; M = 64 at d = 64)
+// dV, dK accumulate in TMEM [256, 256 + d) and [256 + d, 256 + 2 d).
+//
+// The softmax-grad work is split in two phases so that both overlap products:
+//   A(i): P^T from S^T and LSE     (overlaps dK, dQ^T of the previous tile)
+//   B(i): dS^T from dP^T, P and D  (overlaps dV(i) and S^T of the next tile)
+// MMA issue order per tile i (i' = next kept tile):
+//   [P(i) ready] dV(i), S^T(i') | [dS(i) ready] dK(i), dQ^T(i) |
+//   [dQ^T(i) read out] dP^T(i')
+// The tensor pipe completes in issue order, so S^T(i') may overwrite P^T(i)
+// after dV(i), and dP^T(i') completing implies dK(i), dQ^T(i) have finished
+// reading dS^T(i): one dS^T buffer suffices.
+//
+// Warp roles (512 threads, four warpgroups): warps 0-7 softmax-grad (warp w:
+// TMEM lanes 32 (w % 4).., queries [64 (w / 4), +64)), then the dV / dK
+// epilogue; warps 8-11 dQ drain (TMEM -> registers -> fp32 atomics into the
+// accumulator); warp 12 TMA producer; warp 13 MMA issuer (owns TMEM); warps
+// 14-15 idle.  The last warpgroup gives registers to the first three
+// (setmaxnreg: 3 x 128 x 144 + 128 x 80 = 65536).
+// ---------------------------------------------------------------------------
+template <int D, int NS>
 struct BwdCfg {
-    static constexpr int DH = D / DSPLIT;                 // output columns per CTA
-    static constexpr int kKVTile = 128 * D * 2;           // K_j or V_j
-    static constexpr int kKVChunk = 128 * 128;            // 64 columns of a 128-row tile
-    static constexpr int kQTile = BM * D * 2;             // Q_i or dO_i
-    static constexpr int kQChunk = BM * 128;              // 64 columns of a BM-row tile
-    static constexpr int kPTile = 128 * BM * 2;           // P^T or dS^T: 128 keys x BM queries
+    static constexpr int BM = 128;                      // query rows per tile
+    static constexpr int kKVTile = 128 * D * 2;         // K_j or V_j
+    static constexpr int kChunk = 128 * 128;            // 64 columns of a 128-row tile (one swizzle atom wide)
+    static constexpr int kQTile = BM * D * 2;           // Q_i or dO_i
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKOff + kKVTile;
     static constexpr int kQOff = kVOff + kKVTile;
     static constexpr int kdOOff = kQOff + NS * kQTile;
-    static constexpr int kdSOff = kdOOff + NS * kQTile;   // NPB buffers of dS^T
-    static constexpr int kStatOff = kdSOff + NPB * kPTile;   // per stage: lse*log2e [BM], D [BM]
-    static constexpr int kBarOff = kStatOff + NS * BM * 8;
+    static constexpr int kdSOff = kdOOff + NS * kQTile;   // dS^T: [2 query chunks][128 keys][64 queries]
+    static constexpr int kStatBytes = BM * 4;
+    static constexpr int kStatOff = kdSOff + 2 * kChunk;  // per stage: LSE log2 e [BM], D [BM]
+    static constexpr int kBarOff = kStatOff + NS * 2 * kStatBytes;
     static constexpr int kBarKV = 0;
     static constexpr int kBarQFull = 1;
     static constexpr int kBarQEmpty = kBarQFull + NS;
-    static constexpr int kBarSdpFull = kBarQEmpty + NS;
-    static constexpr int kBarSdpEmpty = kBarSdpFull + 1;
-    static constexpr int kBarDsFull = kBarSdpEmpty + 1;
-    static constexpr int kBarPdsEmpty = kBarDsFull + 1;   // NPB barriers, one per P/dS buffer
-    static constexpr int kBarDqFull = kBarPdsEmpty + NPB;
-    static constexpr int kBarDqEmpty = kBarDqFull + 1;
-    static constexpr int kBarMmaDone = kBarDqEmpty + 1;
+    static constexpr int kBarSFull = kBarQEmpty + NS;     // S^T computed
+    static constexpr int kBarDPFull = kBarSFull + 1;      // dP^T computed
+    static constexpr int kBarPFull = kBarDPFull + 1;      // P^T in TMEM (256 arrivals)
+    static constexpr int kBarDsFull = kBarPFull + 1;      // dS^T in smem, dP^T read (256 arrivals)
+    static constexpr int kBarDqFull = kBarDsFull + 1;     // dQ^T computed
+    static constexpr int kBarDqFree = kBarDqFull + 1;     // dQ^T read out (128 arrivals)
+    static constexpr int kBarMmaDone = kBarDqFree + 1;
     static constexpr int kNumBars = kBarMmaDone + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
-    static constexpr int kThreads = 320;
+    // No alignment slack: the kernel checks that dynamic shared memory starts
+    // on a 1 KB boundary (the 128-byte swizzle atoms need it).
+    static constexpr int kSmemBytes = kMiscOff + 16;
+    static constexpr int kThreads = 512;
+    static constexpr int kRegsWork = 144;               // warpgroups 0-2 after setmaxnreg
+    static constexpr int kRegsCtl = 80;                  // warpgroup 3
+    static_assert(3 * 128 * kRegsWork + 128 * kRegsCtl <= 65536, "register split");
+    static constexpr int kWarpTma = 12;
+    static constexpr int kWarpMma = 13;
     static constexpr int kColS = 0;
     static constexpr int kColDP = 128;
     static constexpr int kColDV = 256;
-    static constexpr int kColDK = 256 + DH;
-    static constexpr int kColDQ = DQT ? 64 : 256 + 2 * DH;
-    static constexpr int kDqCols = DQT ? BM : DH;         // fp32 columns per drain thread
-    static constexpr int kColPT = DQT ? 192 : 448;        // NPB buffers of 16-bit P^T (BM / 2 columns each)
-    static constexpr int kStatBytes = BM * 4;
-    static_assert(kColPT + NPB * BM / 2 <= (DQT ? 256 : 512), "P^T columns");
-    static_assert(DQT ? (BM == 64 && DH == 128) : (BM == 128 && DH == 64), "tile shape");
-    static_assert(kColDQ + kDqCols <= 512 && kColDK + DH <= 512, "TMEM columns");
-    static_assert(NPB == 1 || NPB == 2, "P/dS buffers");
+    static constexpr int kColDK = 256 + D;
+    static_assert(D == 64 || D == 128, "head dim");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16>
-__global__ void __launch_bounds__(320, 1)
+constexpr int kErrSmemAlign = 5;   // matches FA_ERR_CUDA
+
+template <int D, int NS, bool BF16>
+__global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
                const BwdParams p) {
-    using C = BwdCfg<D, BM, DSPLIT, NS, NPB, DQT>;
-    constexpr int DH = C::DH;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    using C = BwdCfg<D, NS>;
+    constexpr int BM = C::BM;
+    extern __shared__ __align__(1024) uint8_t smem_buf[];
+    if (smem_u32(smem_buf) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(&g_dev_status, 0, kErrSmemAlign);
+        return;
+    }
+    uint8_t *smem = smem_buf;
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int j = blockIdx.x / DSPLIT;
-    const int h = blockIdx.x % DSPLIT;
-    const int bh = blockIdx.y;
+    const int bh = blockIdx.x;
+    const int j = blockIdx.y;       // key block; causal: the heaviest (j = 0) are scheduled first
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -208,21 +241,21 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar(C::kBarQFull + s), 1);
             mbar_init(bar(C::kBarQEmpty + s), 1);
         }
-        mbar_init(bar(C::kBarSdpFull), 1);
-        mbar_init(bar(C::kBarSdpEmpty), 128);
-        mbar_init(bar(C::kBarDsFull), 128);
-        for (int b = 0; b < NPB; ++b) mbar_init(bar(C::kBarPdsEmpty + b), 1);
+        mbar_init(bar(C::kBarSFull), 1);
+        mbar_init(bar(C::kBarDPFull), 1);
+        mbar_init(bar(C::kBarPFull), 256);
+        mbar_init(bar(C::kBarDsFull), 256);
         mbar_init(bar(C::kBarDqFull), 1);
-        mbar_init(bar(C::kBarDqEmpty), 128);
+        mbar_init(bar(C::kBarDqFree), 128);
         mbar_init(bar(C::kBarMmaDone), 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 9) {
+    if (warp == C::kWarpMma) {
         tmem_alloc(smem_u32(tmem_holder), 512);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == C::kWarpTma && lane == 0) {
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmq);
@@ -235,320 +268,306 @@ __global__ void __launch_bounds__(320, 1)
     int cnt = 0;        // query tiles processed by this warp's role
     bool ok = true;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVTile);
-            for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(sbase + C::kKOff + c * C::kKVChunk, &tmk, bar(C::kBarKV), c * 64, j * 128, bh);
-                tma_load_3d(sbase + C::kVOff + c * C::kKVChunk, &tmv, bar(C::kBarKV), c * 64, j * 128, bh);
-            }
-        }
-        __syncwarp();
-        QIter<BM> it;
-        int i;
-        while (it.next(p, j, i)) {
-            const int s = cnt % NS;
-            const uint32_t ph = (cnt / NS) & 1;
-            ok = wait_bar(bar(C::kBarQEmpty + s), ph ^ 1u, abort_flag);
-            if (!ok) break;
-            // Q_i, dO_i (TMA tiles) and the padded per-row statistics (bulk
-            // copies, prepared by bwd_pre) land on one transaction barrier
+    if (warp >= 12) {
+        setmaxnreg_dec<C::kRegsCtl>();
+        if (warp == C::kWarpTma) {
+            // ------------------------------------------------------------ producer
             if (lane == 0) {
-                const uint32_t qb = bar(C::kBarQFull + s);
-                mbar_arrive_expect_tx(qb, 2 * C::kQTile + 2 * C::kStatBytes);
+                mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVTile);
                 for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, qb, c * 64, i * BM, bh);
-                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo, qb, c * 64, i * BM, bh);
+                    tma_load_3d(sbase + C::kKOff + c * C::kChunk, &tmk, bar(C::kBarKV), c * 64, j * 128, bh);
+                    tma_load_3d(sbase + C::kVOff + c * C::kChunk, &tmv, bar(C::kBarKV), c * 64, j * 128, bh);
                 }
-                const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
-                bulk_load(sbase + C::kStatOff + s * 2 * C::kStatBytes, p.lse2 + srow, C::kStatBytes, qb);
-                bulk_load(sbase + C::kStatOff + s * 2 * C::kStatBytes + C::kStatBytes, p.dvec + srow,
-                          C::kStatBytes, qb);
             }
             __syncwarp();
-            ++cnt;
-        }
-        drain_bar(bar(C::kBarKV), 0);
-        for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
-    } else if (warp == 9) {
-        // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t kIdS = instr_desc_f16(128, BM, BF16, false, false);
-        constexpr uint32_t kIdKV = instr_desc_f16(128, DH, BF16, false, true);
-        constexpr uint32_t kIdQ = DQT ? instr_desc_f16(128, BM, BF16, true, true)
-                                      : instr_desc_f16(128, DH, BF16, true, true);
-        // descriptors built once; each instruction only offsets the start address
-        const SmemDesc dK_kmaj = make_desc(sbase + C::kKOff, 16, 1024);
-        const SmemDesc dV_kmaj = make_desc(sbase + C::kVOff, 16, 1024);
-        const SmemDesc dQ_kmaj = make_desc(sbase + C::kQOff, 16, 1024);
-        const SmemDesc ddO_kmaj = make_desc(sbase + C::kdOOff, 16, 1024);
-        const SmemDesc dQ_mn = make_desc(sbase + C::kQOff + h * (DH / 64) * C::kQChunk, C::kQChunk, 1024);
-        const SmemDesc ddO_mn = make_desc(sbase + C::kdOOff + h * (DH / 64) * C::kQChunk, C::kQChunk, 1024);
-        const SmemDesc ddS_kmaj = make_desc(sbase + C::kdSOff, 16, 1024);
-        const SmemDesc ddS_mn = make_desc(sbase + C::kdSOff, 128 * 128, 1024);
-        const SmemDesc dK_mn = make_desc(sbase + C::kKOff + h * (DH / 64) * C::kKVChunk, C::kKVChunk, 1024);
-        auto issue_sdp = [&](int s) {
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
-                const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColS, dK_kmaj.at(okv), dQ_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
-                const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColDP, dV_kmaj.at(okv), ddO_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
-            }
-        };
-        auto issue_dvdk = [&](int s, int pb, bool acc) {
-#pragma unroll
-            for (int k = 0; k < BM / 16; ++k)   // dV += P^T dO_i, P^T read from TMEM
-                mma_ts(tmem + C::kColDV, tmem + C::kColPT + pb * (BM / 2) + 8 * k,
-                       ddO_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u);
-#pragma unroll
-            for (int k = 0; k < BM / 16; ++k) {
-                const uint32_t oa = pb * C::kPTile + (k >> 2) * (128 * 128) + (k & 3) * 32;
-                mma_ss(tmem + C::kColDK, ddS_kmaj.at(oa), dQ_mn.at(s * C::kQTile + k * 2048), kIdKV,
-                       (acc || k > 0) ? 1u : 0u);
-            }
-        };
-        auto issue_dq = [&](int pb) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if constexpr (DQT) {
-                    // dQ^T (DH x BM) = K_j^T (DH x 128 keys) * dS^T (128 keys x BM)
-                    mma_ss(tmem + C::kColDQ, dK_mn.at(k * 2048), ddS_mn.at(pb * C::kPTile + k * 2048), kIdQ,
-                           k > 0 ? 1u : 0u);
-                } else {
-                    // dQ (BM x DH) = dS (BM x 128 keys) * K_j (128 keys x DH)
-                    mma_ss(tmem + C::kColDQ, ddS_mn.at(pb * C::kPTile + k * 2048), dK_mn.at(k * 2048), kIdQ,
-                           k > 0 ? 1u : 0u);
-                }
-            }
-        };
-
-        QIter<BM> it;
-        int i, in;
-        bool have = it.next(p, j, i);
-        if (have) {
-            ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
+            QIter<BM> it;
+            int i;
+            while (it.next(p, j, i)) {
+                const int s = cnt % NS;
+                ok = wait_bar(bar(C::kBarQEmpty + s), ((cnt / NS) & 1) ^ 1u, abort_flag);
+                if (!ok) break;
+                // Q_i, dO_i (TMA tiles) and the padded per-row statistics (bulk
+                // copies, prepared by bwd_pre) land on one transaction barrier
                 if (lane == 0) {
-                    issue_sdp(0);
-                    mma_commit(bar(C::kBarSdpFull));
+                    const uint32_t qb = bar(C::kBarQFull + s);
+                    mbar_arrive_expect_tx(qb, 2 * C::kQTile + 2 * C::kStatBytes);
+                    for (int c = 0; c < D / 64; ++c) {
+                        tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kChunk, &tmq, qb, c * 64, i * BM, bh);
+                        tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kChunk, &tmdo, qb, c * 64, i * BM, bh);
+                    }
+                    const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
+                    const uint32_t st = sbase + C::kStatOff + s * 2 * C::kStatBytes;
+                    bulk_load(st, p.lse2 + srow, C::kStatBytes, qb);
+                    bulk_load(st + C::kStatBytes, p.dvec + srow, C::kStatBytes, qb);
                 }
                 __syncwarp();
+                ++cnt;
             }
-        }
-        // S^T, dP^T of the next tile: needs the softmax-grad warps to have read
-        // this tile's and the producer to have landed the next Q_i, dO_i
-        auto prefetch_next = [&]() -> bool {
-            const int sn = (cnt + 1) % NS;
-            if (!(wait_bar(bar(C::kBarSdpEmpty), cnt & 1, abort_flag) &&
-                  wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag)))
-                return false;
-            tc_fence_after();
-            if (lane == 0) {
-                issue_sdp(sn);
-                mma_commit(bar(C::kBarSdpFull));
-            }
-            __syncwarp();
-            return true;
-        };
-        while (ok && have) {
-            const int s = cnt % NS;
-            const int pb = cnt % NPB;
-            const bool have_n = it.next(p, j, in);
-            // with two or more stages the next tile is already resident: overlap
-            // its S^T, dP^T with this tile's softmax-grad work.  With one stage
-            // the next tile can only land after this tile's products finish.
-            if (NS >= 2 && have_n) {
-                ok = prefetch_next();
-                if (!ok) break;
-            }
-            ok = wait_bar(bar(C::kBarDsFull), cnt & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) issue_dvdk(s, pb, cnt > 0);
-            __syncwarp();
-            ok = wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-                issue_dq(pb);
-                mma_commit(bar(C::kBarDqFull));
-                mma_commit(bar(C::kBarPdsEmpty + pb));
-                mma_commit(bar(C::kBarQEmpty + s));
-            }
-            __syncwarp();
-            if (NS == 1 && have_n) {
-                ok = prefetch_next();
-                if (!ok) break;
-            }
-            ++cnt;
-            have = have_n;
-            i = in;
-        }
-        if (lane == 0) mma_commit(bar(C::kBarMmaDone));
-        __syncwarp();
-        drain_bar(bar(C::kBarMmaDone), 0);
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ softmax-grad
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const int r = warp * 32 + lane;     // key row within the block
-        const int key = j * 128 + r;
-        const float c = p.scale_log2;
-        QIter<BM> it;
-        int i;
-        while (it.next(p, j, i)) {
-            const int s = cnt % NS;
-            const int pb = cnt % NPB;
-            uint8_t *sdS = smem + C::kdSOff + pb * C::kPTile;
-            const uint32_t tP = tmem + lane_off + C::kColPT + pb * (BM / 2);
-            ok = wait_bar(bar(C::kBarSdpFull), cnt & 1, abort_flag) &&
-                 wait_bar(bar(C::kBarQFull + s), (cnt / NS) & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
-            const float4 *dd4 = lse4 + BM / 4;
-            const bool need_causal = (p.mode & kCausal) && (i * BM < j * 128 + 127);
-#pragma unroll 1
-            for (int ch = 0; ch < BM / 32; ++ch) {
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tmem + lane_off + C::kColS + 32 * ch, sr);
-                tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, pr);
-                tmem_ld_wait();
-                if (ch == BM / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(bar(C::kBarSdpEmpty));
+            drain_bar(bar(C::kBarKV), 0);
+            for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
+        } else if (warp == C::kWarpMma) {
+            // ------------------------------------------------------------ MMA issuer
+            constexpr uint32_t kIdS = instr_desc_f16(128, BM, BF16, false, false);   // S^T, dP^T
+            constexpr uint32_t kIdKV = instr_desc_f16(128, D, BF16, false, true);    // dV, dK
+            constexpr uint32_t kIdQ = instr_desc_f16(D, BM, BF16, true, true);       // dQ^T
+            // descriptors built once; each instruction only offsets the start address
+            const SmemDesc dK_k = make_desc(sbase + C::kKOff, 16, 1024);
+            const SmemDesc dV_k = make_desc(sbase + C::kVOff, 16, 1024);
+            const SmemDesc dQ_k = make_desc(sbase + C::kQOff, 16, 1024);
+            const SmemDesc ddO_k = make_desc(sbase + C::kdOOff, 16, 1024);
+            const SmemDesc dQ_mn = make_desc(sbase + C::kQOff, C::kChunk, 1024);
+            const SmemDesc ddO_mn = make_desc(sbase + C::kdOOff, C::kChunk, 1024);
+            const SmemDesc ddS_k = make_desc(sbase + C::kdSOff, 16, 1024);
+            const SmemDesc ddS_mn = make_desc(sbase + C::kdSOff, C::kChunk, 1024);
+            const SmemDesc dK_mn = make_desc(sbase + C::kKOff, C::kChunk, 1024);
+            auto issue_s = [&](int s) {          // S^T = K_j Q_i^T
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t o = (k >> 2) * C::kChunk + (k & 3) * 32;
+                    mma_ss(tmem + C::kColS, dK_k.at(o), dQ_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u);
                 }
-                uint32_t pk[16], dk[16];
+            };
+            auto issue_dp = [&](int s) {         // dP^T = V_j dO_i^T
 #pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    const float4 l4 = lse4[ch * 8 + k4];
-                    const float4 d4 = dd4[ch * 8 + k4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pp[4], ds[4];
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t o = (k >> 2) * C::kChunk + (k & 3) * 32;
+                    mma_ss(tmem + C::kColDP, dV_k.at(o), ddO_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_dv = [&](int s, bool acc) {   // dV += P^T dO_i; P^T of queries 16k.. at column 8k + 32 (k / 4)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int kk = 4 * k4 + e;
-                        float pv = ex2(fmaf(__uint_as_float(sr[kk]), c, -lv[e]));
-                        if (need_causal && key > i * BM + 32 * ch + kk) pv = 0.f;
-                        pp[e] = pv;
-                        ds[e] = pv * (__uint_as_float(pr[kk]) - dv[e]);
+                for (int k = 0; k < BM / 16; ++k)
+                    mma_ts(tmem + C::kColDV, tmem + C::kColS + 8 * k + 32 * (k >> 2), ddO_mn.at(s * C::kQTile + k * 2048),
+                           kIdKV, (acc || k > 0) ? 1u : 0u);
+            };
+            auto issue_dk_dq = [&](int s, bool acc) {
+#pragma unroll
+                for (int k = 0; k < BM / 16; ++k)    // dK += dS^T Q_i
+                    mma_ss(tmem + C::kColDK, ddS_k.at((k >> 2) * C::kChunk + (k & 3) * 32),
+                           dQ_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)          // dQ^T (D x BM) = K_j^T dS^T, over the 128 keys
+                    mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u);
+            };
+
+            QIter<BM> it;
+            int i, in;
+            bool have = it.next(p, j, i);
+            if (have) {
+                ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_s(0);
+                        mma_commit(bar(C::kBarSFull));
+                        issue_dp(0);
+                        mma_commit(bar(C::kBarDPFull));
                     }
-                    pk[2 * k4] = pack2<BF16>(pp[0], pp[1]);
-                    pk[2 * k4 + 1] = pack2<BF16>(pp[2], pp[3]);
-                    dk[2 * k4] = pack2<BF16>(ds[0], ds[1]);
-                    dk[2 * k4 + 1] = pack2<BF16>(ds[2], ds[3]);
-                }
-                if (ch == 0 && cnt >= NPB) {
-                    // the products that read this P/dS buffer NPB tiles ago must be done
-                    if (!wait_bar(bar(C::kBarPdsEmpty + pb), ((cnt / NPB) - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                // P^T row r -> TMEM (A operand of dV); dS^T row r -> a K-major
-                // [BM/64][128][64] 128B-swizzled shared tile (dK and dQ operand)
-                tmem_st16(tP + 16 * ch, pk);
-                const int chunk = (32 * ch) / 64;
-                const int u0 = ((32 * ch) % 64) / 8;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int off = chunk * (128 * 128) + r * 128 + (((u0 + u) ^ (r & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(sdS + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+                    __syncwarp();
                 }
             }
-            if (!ok) break;
-            tmem_st_wait();
-            tc_fence_before();
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(bar(C::kBarDsFull));
-            ++cnt;
+            while (ok && have) {
+                const int s = cnt % NS;
+                const int sn = (cnt + 1) % NS;
+                const uint32_t ph = cnt & 1;
+                const bool have_n = it.next(p, j, in);
+                ok = wait_bar(bar(C::kBarPFull), ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) issue_dv(s, cnt > 0);
+                __syncwarp();
+                if (have_n) {
+                    ok = wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_s(sn);
+                        mma_commit(bar(C::kBarSFull));
+                    }
+                    __syncwarp();
+                }
+                ok = wait_bar(bar(C::kBarDsFull), ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_dk_dq(s, cnt > 0);
+                    mma_commit(bar(C::kBarDqFull));
+                    mma_commit(bar(C::kBarQEmpty + s));
+                }
+                __syncwarp();
+                if (have_n) {
+                    ok = wait_bar(bar(C::kBarDqFree), ph, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_dp(sn);
+                        mma_commit(bar(C::kBarDPFull));
+                    }
+                    __syncwarp();
+                }
+                ++cnt;
+                have = have_n;
+                i = in;
+            }
+            if (lane == 0) mma_commit(bar(C::kBarMmaDone));
+            __syncwarp();
+            drain_bar(bar(C::kBarMmaDone), 0);
         }
     } else {
-        // ------------------------------------------------------------ dQ drain
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const int t = (warp & 3) * 32 + lane;   // TMEM lane: a d index (transposed form) or a query row
-        QIter<BM> it;
-        int i;
-        while (it.next(p, j, i)) {
-            ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t v[C::kDqCols];
+        setmaxnreg_inc<C::kRegsWork>();
+        if (warp < 8) {
+            // ------------------------------------------------------------ softmax-grad
+            const int qd = warp & 3;            // TMEM lane quadrant
+            const int qh = warp >> 2;           // query half
+            const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+            const int r = qd * 32 + lane;       // key row within the block
+            const float c = p.scale_log2;
+            QIter<BM> it;
+            int i;
+            while (it.next(p, j, i)) {
+                const int s = cnt % NS;
+                const uint32_t ph = cnt & 1;
+                ok = wait_bar(bar(C::kBarSFull), ph, abort_flag) &&
+                     wait_bar(bar(C::kBarQFull + s), (cnt / NS) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
+                const float4 *dd4 = lse4 + BM / 4;
+                const bool diag = (p.mode & kCausal) && i == j;
+                // phase A: P^T = 2^(S^T * scale * log2 e - LSE * log2 e), masked
+                float pv[64];
 #pragma unroll
-            for (int ch = 0; ch < C::kDqCols / 32; ++ch)
-                tmem_ld32(tmem + lane_off + C::kColDQ + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarDqEmpty));
-            float *accb = p.dqacc + static_cast<size_t>(bh) * p.N * D;
-            if constexpr (DQT) {
-                const int dcol = h * DH + t;
-#pragma unroll
-                for (int k = 0; k < BM; ++k) {
-                    const int q = i * BM + k;
-                    if (q < p.N) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
-                }
-            } else {
-                const int q = i * BM + t;
-                if (q < p.N) {
-                    float4 *dst = reinterpret_cast<float4 *>(accb + static_cast<size_t>(q) * D + h * DH);
-#pragma unroll
-                    for (int k = 0; k < DH / 4; ++k)
-                        atomicAdd(dst + k, make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                                       __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3])));
-                }
-            }
-            ++cnt;
-        }
-    }
-
-    // ---------------------------------------------------------------- dV / dK epilogue
-    if (warp < 8) {
-        bool done = ok;
-        if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
-        tc_fence_after();
-        const bool is_dv = warp < 4;
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const int r = (warp & 3) * 32 + lane;
-        const int key = j * 128 + r;
-        const float mul = is_dv ? 1.0f : p.scale;
-        uint8_t *out = reinterpret_cast<uint8_t *>(is_dv ? p.dv : p.dk);
-        const uint32_t col0 = is_dv ? C::kColDV : C::kColDK;
-        if (done) {
-#pragma unroll 1
-            for (int ch = 0; ch < DH / 32; ++ch) {
-                uint32_t v[32];
-                if (cnt > 0) {
-                    tmem_ld32(tmem + lane_off + col0 + 32 * ch, v);
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int q0 = 64 * qh + 32 * ch;
+                    uint32_t sr[32];
+                    tmem_ld32(tmem + lane_off + C::kColS + q0, sr);
                     tmem_ld_wait();
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = 0u;
-                }
-                if (key < p.N) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D +
-                                                                  h * DH + 32 * ch) * 2);
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        const float4 l4 = lse4[q0 / 4 + k4];
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int kk = 4 * k4 + e;
+                            float x = ex2(fmaf(__uint_as_float(sr[kk]), c, -lv[e]));
+                            if (diag && r > q0 + kk) x = 0.f;
+                            pv[32 * ch + kk] = x;
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) pk[k] = pack2<BF16>(pv[32 * ch + 2 * k], pv[32 * ch + 2 * k + 1]);
+                    // 16-bit P^T of queries q0.. over S^T columns already read
+                    tmem_st16(tmem + lane_off + C::kColS + 64 * qh + 16 * ch, pk);
                 }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull));
+                // phase B: dS^T = P^T o (dP^T - D)
+                ok = wait_bar(bar(C::kBarDPFull), ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                uint8_t *sdS = smem + C::kdSOff + qh * C::kChunk + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int q0 = 64 * qh + 32 * ch;
+                    uint32_t pr[32];
+                    tmem_ld32(tmem + lane_off + C::kColDP + q0, pr);
+                    tmem_ld_wait();
+                    uint32_t dk[16];
+#pragma unroll
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        const float4 d4 = dd4[q0 / 4 + k4];
+                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float ds[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) ds[e] = pv[32 * ch + 4 * k4 + e] * (__uint_as_float(pr[4 * k4 + e]) - dv[e]);
+                        dk[2 * k4] = pack2<BF16>(ds[0], ds[1]);
+                        dk[2 * k4 + 1] = pack2<BF16>(ds[2], ds[3]);
+                    }
+                    // row r of a K-major [128 keys][64 queries] 128B-swizzled tile
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int off = ((4 * ch + u) ^ (r & 7)) << 4;
+                        *reinterpret_cast<uint4 *>(sdS + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+                    }
+                }
+                tc_fence_before();
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(bar(C::kBarDsFull));
+                ++cnt;
+            }
+            // ------------------------------------------------------------ dV / dK epilogue
+            {
+                bool done = ok;
+                if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
+                tc_fence_after();
+                const bool is_dv = warp < 4;
+                const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+                const int r = (warp & 3) * 32 + lane;
+                const int key = j * 128 + r;
+                const float mul = is_dv ? 1.0f : p.scale;
+                uint8_t *out = reinterpret_cast<uint8_t *>(is_dv ? p.dv : p.dk);
+                const uint32_t col0 = is_dv ? C::kColDV : C::kColDK;
+                if (done) {
+        #pragma unroll 1
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t v[32];
+                        if (cnt > 0) {
+                            tmem_ld32(tmem + lane_off + col0 + 32 * ch, v);
+                            tmem_ld_wait();
+                        } else {
+        #pragma unroll
+                            for (int k = 0; k < 32; ++k) v[k] = 0u;
+                        }
+                        if (key < p.N) {
+                            uint32_t pk[16];
+        #pragma unroll
+                            for (int k = 0; k < 16; ++k)
+                                pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+                            uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D + 32 * ch) * 2);
+        #pragma unroll
+                            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                        }
+                    }
+                }
+            }
+        } else {
+            // ------------------------------------------------------------ dQ drain
+            // dQ^T rows are d indices.  At d = 128 every TMEM lane is a row; at
+            // d = 64 (an M = 64 product) row m sits in lane 32 (m / 16) + m % 16.
+            const int wq = warp & 3;
+            const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+            const bool row_lane = (D == 128) || (lane < 16);
+            const int dcol = (D == 128) ? wq * 32 + lane : wq * 16 + (lane & 15);
+            QIter<BM> it;
+            int i;
+            while (it.next(p, j, i)) {
+                ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t v[BM];
+#pragma unroll
+                for (int ch = 0; ch < BM / 32; ++ch)
+                    tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarDqFree));
+                if (row_lane) {
+                    float *acc = p.dqacc + (static_cast<size_t>(bh) * p.N + static_cast<size_t>(i) * BM) * D + dcol;
+                    const int lim = p.N - i * BM;
+#pragma unroll
+                    for (int k = 0; k < BM; ++k)
+                        if (k < lim) atomicAdd(acc + k * D, __uint_as_float(v[k]));
+                }
+                ++cnt;
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == C::kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -273,6 +273,17 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(int M, int N, bool bf16, b
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Register reallocation between warpgroups (every warp of a warpgroup
+// executes the same one; the counts are multiples of 8).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------
 // math
 // ---------------------------------------------------------------------------
