@@ -434,62 +434,61 @@ __global__ void __launch_bounds__(512, 1)
                 const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
                 const float4 *dd4 = lse4 + BM / 4;
                 const bool diag = (p.mode & kCausal) && i == j;
-                // phase A: P^T = 2^(S^T * scale * log2 e - LSE * log2 e), masked
-                float pv[64];
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int q0 = 64 * qh + 32 * ch;
-                    uint32_t sr[32];
-                    tmem_ld32(tmem + lane_off + C::kColS + q0, sr);
+                // phase A: P^T = 2^(S^T * scale * log2 e - LSE * log2 e), masked,
+                // rounded to 16 bits (kept packed in registers for phase B) and
+                // written over the S^T columns already read
+                const int q0 = 64 * qh;
+                uint32_t pk[32];
+                {
+                    uint32_t sr[64];
+                    tmem_ld32(tmem + lane_off + C::kColS + q0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld32(tmem + lane_off + C::kColS + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                     tmem_ld_wait();
-                    uint32_t pk[16];
+                    const int lim = diag ? r - q0 : -1;    // queries q0 + kk with kk < lim precede key r
 #pragma unroll
-                    for (int k4 = 0; k4 < 8; ++k4) {
+                    for (int k4 = 0; k4 < 16; ++k4) {
                         const float4 l4 = lse4[q0 / 4 + k4];
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int kk = 4 * k4 + e;
-                            float x = ex2(fmaf(__uint_as_float(sr[kk]), c, -lv[e]));
-                            if (diag && r > q0 + kk) x = 0.f;
-                            pv[32 * ch + kk] = x;
-                        }
+                        float x0 = ex2(fmaf(__uint_as_float(sr[4 * k4]), c, -l4.x));
+                        float x1 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 1]), c, -l4.y));
+                        float x2 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 2]), c, -l4.z));
+                        float x3 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 3]), c, -l4.w));
+                        if (4 * k4 < lim) x0 = 0.f;
+                        if (4 * k4 + 1 < lim) x1 = 0.f;
+                        if (4 * k4 + 2 < lim) x2 = 0.f;
+                        if (4 * k4 + 3 < lim) x3 = 0.f;
+                        pk[2 * k4] = pack2<BF16>(x0, x1);
+                        pk[2 * k4 + 1] = pack2<BF16>(x2, x3);
                     }
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) pk[k] = pack2<BF16>(pv[32 * ch + 2 * k], pv[32 * ch + 2 * k + 1]);
-                    // 16-bit P^T of queries q0.. over S^T columns already read
-                    tmem_st16(tmem + lane_off + C::kColS + 64 * qh + 16 * ch, pk);
                 }
+                tmem_st32(tmem + lane_off + C::kColS + q0, pk);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarPFull));
-                // phase B: dS^T = P^T o (dP^T - D)
+                // phase B: dS^T = P^T o (dP^T - D), with the 16-bit P^T
                 ok = wait_bar(bar(C::kBarDPFull), ph, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                uint8_t *sdS = smem + C::kdSOff + qh * C::kChunk + r * 128;
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int q0 = 64 * qh + 32 * ch;
-                    uint32_t pr[32];
-                    tmem_ld32(tmem + lane_off + C::kColDP + q0, pr);
+                {
+                    uint32_t pr[64];
+                    tmem_ld32(tmem + lane_off + C::kColDP + q0, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+                    tmem_ld32(tmem + lane_off + C::kColDP + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
                     tmem_ld_wait();
-                    uint32_t dk[16];
-#pragma unroll
-                    for (int k4 = 0; k4 < 8; ++k4) {
-                        const float4 d4 = dd4[q0 / 4 + k4];
-                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                        float ds[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) ds[e] = pv[32 * ch + 4 * k4 + e] * (__uint_as_float(pr[4 * k4 + e]) - dv[e]);
-                        dk[2 * k4] = pack2<BF16>(ds[0], ds[1]);
-                        dk[2 * k4 + 1] = pack2<BF16>(ds[2], ds[3]);
-                    }
                     // row r of a K-major [128 keys][64 queries] 128B-swizzled tile
+                    uint8_t *sdS = smem + C::kdSOff + qh * C::kChunk + r * 128;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int off = ((4 * ch + u) ^ (r & 7)) << 4;
-                        *reinterpret_cast<uint4 *>(sdS + off) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+                    for (int u = 0; u < 8; ++u) {
+                        uint32_t dk[4];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const int k4 = 2 * u + h2;
+                            const float4 d4 = dd4[q0 / 4 + k4];
+                            const float2 p01 = unpack2<BF16>(pk[2 * k4]), p23 = unpack2<BF16>(pk[2 * k4 + 1]);
+                            dk[2 * h2] = pack2<BF16>(p01.x * (__uint_as_float(pr[4 * k4]) - d4.x),
+                                                     p01.y * (__uint_as_float(pr[4 * k4 + 1]) - d4.y));
+                            dk[2 * h2 + 1] = pack2<BF16>(p23.x * (__uint_as_float(pr[4 * k4 + 2]) - d4.z),
+                                                         p23.y * (__uint_as_float(pr[4 * k4 + 3]) - d4.w));
+                        }
+                        *reinterpret_cast<uint4 *>(sdS + ((u ^ (r & 7)) << 4)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
                     }
                 }
                 tc_fence_before();

@@ -201,6 +201,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -307,8 +318,8 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 template <bool BF16>
 __device__ __forceinline__ float2 unpack2(uint32_t u) {
     if constexpr (BF16) {
-        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u);
-        return __bfloat1622float2(h);
+        // a bf16 is the top half of the fp32 with the same value
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
     } else {
         __half2 h = *reinterpret_cast<__half2 *>(&u);
         return __half22float2(h);
