@@ -91,19 +91,19 @@ int check_common(int B, int H, int N, int d, float scale, int dtype) {
     if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     const long long BH = static_cast<long long>(B) * H;
     if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-    // grid.y holds query-block pairs (<= 65535)
-    if ((static_cast<long long>(N) + 255) / 256 > 65535) return FA_ERR_UNSUPPORTED;
     return FA_OK;
 }
 
-template <int D, int NQ, int NS, bool BF16>
+template <int D, int NQ, int NSK, int NSV, bool BF16>
 int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const fa::FwdParams &p,
                int BH, cudaStream_t stream) {
-    using C = fa::FwdCfg<D, NQ, NS>;
-    auto kern = fa::fwd_kernel<D, NQ, NS, BF16>;
+    using C = fa::FwdCfg<D, NQ, NSK, NSV>;
+    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
-    dim3 grid(BH, (p.nqb + NQ - 1) / NQ);
+    const long long ctas = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
+    if (ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    dim3 grid(static_cast<unsigned>(ctas));
     ProfScope prof(0, stream);
     kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -113,9 +113,9 @@ template <bool BF16>
 int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                  const fa::FwdParams &p, int BH, cudaStream_t s) {
     switch (d) {
-        case 64: return launch_fwd<64, 2, 4, BF16>(mq, mk, mv, p, BH, s);
-        case 128: return launch_fwd<128, 2, 2, BF16>(mq, mk, mv, p, BH, s);
-        case 256: return launch_fwd<256, 1, 1, BF16>(mq, mk, mv, p, BH, s);
+        case 64: return launch_fwd<64, 2, 6, 4, BF16>(mq, mk, mv, p, BH, s);
+        case 128: return launch_fwd<128, 2, 3, 2, BF16>(mq, mk, mv, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, 1, BF16>(mq, mk, mv, p, BH, s);
         default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -128,6 +128,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_MISALIGNED;
     const int BH = B * H;
+    if (static_cast<long long>(BH) * ((N + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // 1-D grid
     CUtensorMap mq, mk, mv;
     if ((rc = make_map(&mq, q, d, N, BH, dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mk, k, d, N, BH, dtype, 128)) != FA_OK) return rc;
@@ -139,6 +140,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     p.N = N;
     p.nqb = (N + 127) / 128;
     p.nkb = p.nqb;
+    p.nbh = BH;
     p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
     p.scale_log2 = scale * kLog2e;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -201,6 +203,7 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, MakeGrid make_grid, con
     p.Npad = Npad;
     p.nkb = (N + 127) / 128;
     p.nqt = (N + BM - 1) / BM;
+    p.nbh = BH;
     p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
@@ -218,10 +221,10 @@ template <bool BF16>
 int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, void *ws, const uint8_t *mask,
                  int BH, int N, float scale, int causal, int dtype, cudaStream_t s) {
-    // d <= 128: grid (BH, key blocks), so that the heaviest causal key blocks
-    // (j = 0) are scheduled first.  d = 256: two CTAs per key block.
-    auto grid_bh_j = [](int nkb, int bh) { return dim3(bh, nkb); };
-    auto grid_split = [](int nkb, int bh) { return dim3(nkb * 2, bh); };
+    // One-dimensional grids of BH x key blocks CTAs (x 2 at d = 256: two CTAs
+    // per key block).
+    auto grid_bh_j = [](int nkb, int bh) { return dim3(static_cast<unsigned>(static_cast<long long>(bh) * nkb)); };
+    auto grid_split = [](int nkb, int bh) { return dim3(static_cast<unsigned>(static_cast<long long>(bh) * nkb * 2)); };
     switch (d) {
         case 64: {
             using C = fa::BwdCfg<64, 3>;
@@ -255,7 +258,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const v
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
     const long long BH = static_cast<long long>(B) * H;
-    if ((N + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;   // key blocks index grid.y
+    if (BH * (2LL * ((N + 127) / 128)) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
     const size_t need = fa::bwd_workspace_bytes(BH, N, d);
     if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FA_ERR_MISALIGNED;

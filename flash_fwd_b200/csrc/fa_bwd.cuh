@@ -46,6 +46,7 @@ struct BwdParams {
     int Npad;             // N rounded up to 128: row pitch of lse2 and dvec
     int nkb;              // key blocks (and mask blocks) of 128
     int nqt;              // query tiles of BM rows
+    int nbh;              // batch x heads
     int mode;
     float scale;
     float scale_log2;
@@ -228,8 +229,10 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
-    const int j = blockIdx.y;       // key block; causal: the heaviest (j = 0) are scheduled first
+    // one-dimensional grid, (batch, head) minor: causal runs the heaviest key
+    // blocks (j = 0) of every (b, h) first (longest work first)
+    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+    const int j = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -307,6 +310,7 @@ __global__ void __launch_bounds__(512, 1)
             for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
         } else if (warp == C::kWarpMma) {
             // ------------------------------------------------------------ MMA issuer
+            const uint32_t leader = elect_one();   // the lane that issues tcgen05 ops
             constexpr uint32_t kIdS = instr_desc_f16(128, BM, BF16, false, false);   // S^T, dP^T
             constexpr uint32_t kIdKV = instr_desc_f16(128, D, BF16, false, true);    // dV, dK
             constexpr uint32_t kIdQ = instr_desc_f16(D, BM, BF16, true, true);       // dQ^T
@@ -324,30 +328,30 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t o = (k >> 2) * C::kChunk + (k & 3) * 32;
-                    mma_ss(tmem + C::kColS, dK_k.at(o), dQ_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColS, dK_k.at(o), dQ_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u, leader);
                 }
             };
             auto issue_dp = [&](int s) {         // dP^T = V_j dO_i^T
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t o = (k >> 2) * C::kChunk + (k & 3) * 32;
-                    mma_ss(tmem + C::kColDP, dV_k.at(o), ddO_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColDP, dV_k.at(o), ddO_k.at(s * C::kQTile + o), kIdS, k > 0 ? 1u : 0u, leader);
                 }
             };
             auto issue_dv = [&](int s, bool acc) {   // dV += P^T dO_i; P^T of queries 16k.. at column 8k + 32 (k / 4)
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)
                     mma_ts(tmem + C::kColDV, tmem + C::kColS + 8 * k + 32 * (k >> 2), ddO_mn.at(s * C::kQTile + k * 2048),
-                           kIdKV, (acc || k > 0) ? 1u : 0u);
+                           kIdKV, (acc || k > 0) ? 1u : 0u, leader);
             };
             auto issue_dk_dq = [&](int s, bool acc) {
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)    // dK += dS^T Q_i
                     mma_ss(tmem + C::kColDK, ddS_k.at((k >> 2) * C::kChunk + (k & 3) * 32),
-                           dQ_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u);
+                           dQ_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u, leader);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)          // dQ^T (D x BM) = K_j^T dS^T, over the 128 keys
-                    mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u, leader);
             };
 
             QIter<BM> it;
@@ -357,11 +361,11 @@ __global__ void __launch_bounds__(512, 1)
                 ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
                 if (ok) {
                     tc_fence_after();
-                    if (lane == 0) {
+                    {
                         issue_s(0);
-                        mma_commit(bar(C::kBarSFull));
+                        mma_commit(bar(C::kBarSFull), leader);
                         issue_dp(0);
-                        mma_commit(bar(C::kBarDPFull));
+                        mma_commit(bar(C::kBarDPFull), leader);
                     }
                     __syncwarp();
                 }
@@ -374,34 +378,34 @@ __global__ void __launch_bounds__(512, 1)
                 ok = wait_bar(bar(C::kBarPFull), ph, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) issue_dv(s, cnt > 0);
+                issue_dv(s, cnt > 0);
                 __syncwarp();
                 if (have_n) {
                     ok = wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    if (lane == 0) {
+                    {
                         issue_s(sn);
-                        mma_commit(bar(C::kBarSFull));
+                        mma_commit(bar(C::kBarSFull), leader);
                     }
                     __syncwarp();
                 }
                 ok = wait_bar(bar(C::kBarDsFull), ph, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) {
+                {
                     issue_dk_dq(s, cnt > 0);
-                    mma_commit(bar(C::kBarDqFull));
-                    mma_commit(bar(C::kBarQEmpty + s));
+                    mma_commit(bar(C::kBarDqFull), leader);
+                    mma_commit(bar(C::kBarQEmpty + s), leader);
                 }
                 __syncwarp();
                 if (have_n) {
                     ok = wait_bar(bar(C::kBarDqFree), ph, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    if (lane == 0) {
+                    {
                         issue_dp(sn);
-                        mma_commit(bar(C::kBarDPFull));
+                        mma_commit(bar(C::kBarDPFull), leader);
                     }
                     __syncwarp();
                 }
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(512, 1)
                 have = have_n;
                 i = in;
             }
-            if (lane == 0) mma_commit(bar(C::kBarMmaDone));
+            mma_commit(bar(C::kBarMmaDone), leader);
             __syncwarp();
             drain_bar(bar(C::kBarMmaDone), 0);
         }
@@ -516,16 +520,16 @@ __global__ void __launch_bounds__(512, 1)
                             tmem_ld32(tmem + lane_off + col0 + 32 * ch, v);
                             tmem_ld_wait();
                         } else {
-        #pragma unroll
+    #pragma unroll
                             for (int k = 0; k < 32; ++k) v[k] = 0u;
                         }
                         if (key < p.N) {
                             uint32_t pk[16];
-        #pragma unroll
+    #pragma unroll
                             for (int k = 0; k < 16; ++k)
                                 pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
                             uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D + 32 * ch) * 2);
-        #pragma unroll
+    #pragma unroll
                             for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                         }
                     }

@@ -70,9 +70,11 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int j = blockIdx.x / DSPLIT;
-    const int h = blockIdx.x % DSPLIT;
-    const int bh = blockIdx.y;
+    // one-dimensional grid, (batch, head) minor (see bwd_kernel)
+    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+    const int jh = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    const int j = jh / DSPLIT;
+    const int h = jh % DSPLIT;
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -149,6 +151,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
+        const uint32_t leader = elect_one();   // the lane that issues tcgen05 ops
         constexpr uint32_t kIdS = instr_desc_f16(128, BM, BF16, false, false);
         constexpr uint32_t kIdKV = instr_desc_f16(128, DH, BF16, false, true);
         constexpr uint32_t kIdQ = DQT ? instr_desc_f16(128, BM, BF16, true, true)
@@ -168,25 +171,25 @@ __global__ void __launch_bounds__(320, 1)
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
                 const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColS, dK_kmaj.at(okv), dQ_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::kColS, dK_kmaj.at(okv), dQ_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u, leader);
             }
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t okv = (k >> 2) * C::kKVChunk + (k & 3) * 32;
                 const uint32_t oq = s * C::kQTile + (k >> 2) * C::kQChunk + (k & 3) * 32;
-                mma_ss(tmem + C::kColDP, dV_kmaj.at(okv), ddO_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::kColDP, dV_kmaj.at(okv), ddO_kmaj.at(oq), kIdS, k > 0 ? 1u : 0u, leader);
             }
         };
         auto issue_dvdk = [&](int s, int pb, bool acc) {
 #pragma unroll
             for (int k = 0; k < BM / 16; ++k)   // dV += P^T dO_i, P^T read from TMEM
                 mma_ts(tmem + C::kColDV, tmem + C::kColPT + pb * (BM / 2) + 8 * k,
-                       ddO_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u);
+                       ddO_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u, leader);
 #pragma unroll
             for (int k = 0; k < BM / 16; ++k) {
                 const uint32_t oa = pb * C::kPTile + (k >> 2) * (128 * 128) + (k & 3) * 32;
                 mma_ss(tmem + C::kColDK, ddS_kmaj.at(oa), dQ_mn.at(s * C::kQTile + k * 2048), kIdKV,
-                       (acc || k > 0) ? 1u : 0u);
+                       (acc || k > 0) ? 1u : 0u, leader);
             }
         };
         auto issue_dq = [&](int pb) {
@@ -195,11 +198,11 @@ __global__ void __launch_bounds__(320, 1)
                 if constexpr (DQT) {
                     // dQ^T (DH x BM) = K_j^T (DH x 128 keys) * dS^T (128 keys x BM)
                     mma_ss(tmem + C::kColDQ, dK_mn.at(k * 2048), ddS_mn.at(pb * C::kPTile + k * 2048), kIdQ,
-                           k > 0 ? 1u : 0u);
+                           k > 0 ? 1u : 0u, leader);
                 } else {
                     // dQ (BM x DH) = dS (BM x 128 keys) * K_j (128 keys x DH)
                     mma_ss(tmem + C::kColDQ, ddS_mn.at(pb * C::kPTile + k * 2048), dK_mn.at(k * 2048), kIdQ,
-                           k > 0 ? 1u : 0u);
+                           k > 0 ? 1u : 0u, leader);
                 }
             }
         };
@@ -211,9 +214,9 @@ __global__ void __launch_bounds__(320, 1)
             ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                if (lane == 0) {
+                {
                     issue_sdp(0);
-                    mma_commit(bar(C::kBarSdpFull));
+                    mma_commit(bar(C::kBarSdpFull), leader);
                 }
                 __syncwarp();
             }
@@ -226,9 +229,9 @@ __global__ void __launch_bounds__(320, 1)
                   wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag)))
                 return false;
             tc_fence_after();
-            if (lane == 0) {
+            {
                 issue_sdp(sn);
-                mma_commit(bar(C::kBarSdpFull));
+                mma_commit(bar(C::kBarSdpFull), leader);
             }
             __syncwarp();
             return true;
@@ -247,16 +250,16 @@ __global__ void __launch_bounds__(320, 1)
             ok = wait_bar(bar(C::kBarDsFull), cnt & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            if (lane == 0) issue_dvdk(s, pb, cnt > 0);
+            issue_dvdk(s, pb, cnt > 0);
             __syncwarp();
             ok = wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            if (lane == 0) {
+            {
                 issue_dq(pb);
-                mma_commit(bar(C::kBarDqFull));
-                mma_commit(bar(C::kBarPdsEmpty + pb));
-                mma_commit(bar(C::kBarQEmpty + s));
+                mma_commit(bar(C::kBarDqFull), leader);
+                mma_commit(bar(C::kBarPdsEmpty + pb), leader);
+                mma_commit(bar(C::kBarQEmpty + s), leader);
             }
             __syncwarp();
             if (NS == 1 && have_n) {
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(320, 1)
             have = have_n;
             i = in;
         }
-        if (lane == 0) mma_commit(bar(C::kBarMmaDone));
+        mma_commit(bar(C::kBarMmaDone), leader);
         __syncwarp();
         drain_bar(bar(C::kBarMmaDone), 0);
     } else if (warp < 4) {

@@ -11,7 +11,10 @@
 //
 // Decomposition (the outer-Q / inner-K/V order of 深度解析 section 四): one
 // CTA owns NQ query tiles of 128 rows of one (batch, head) and streams the
-// kept 128-key tiles of K and V through an NS-stage shared-memory ring.
+// kept 128-key tiles of K and V through shared-memory rings of NSK (K) and
+// NSV (V) stages.  K gets the deeper ring: S of the next key tile is issued
+// right after P V of the current one, so its K tile is needed a whole
+// softmax phase before its V tile.
 //
 // Warp roles (a B200 design; the pages' own schedules target A100/H100):
 //   warps 0 .. 4*NQ-1   softmax: warpgroup t owns query tile t, one thread per
@@ -19,7 +22,9 @@
 //                       rescales O_t in TMEM when m grew by more than 2^8
 //                       (exactness is kept because O and l share the stale m),
 //                       writes P_t (16-bit) back over S_t and signals the MMA warp.
-//   warp 4*NQ           TMA producer: Q tiles once, then K_j and V_j per stage.
+//   warp 4*NQ           TMA producer: Q tiles once, then K_j per stage (and
+//                       V_j when NQ = 1).
+//   warp 4*NQ+2         (NQ = 2) TMA producer of the V_j tiles.
 //   warp 4*NQ+1         MMA issuer (one elected lane): S_t = Q_t K_j^T (SS form)
 //                       and O_t += P_t V_j (P read from TMEM, TS form).  It owns
 //                       the 512-column TMEM allocation.
@@ -28,6 +33,9 @@
 //
 // Scale handling: exp is evaluated as 2^(s * scale * log2 e - m), with the
 // running max m kept in that base-2 domain; LSE converts back to natural log.
+// The exp2 work is split between the special-function unit and the FMA pipe
+// (a degree-3 polynomial for 3 of every 8 pairs), whose throughputs on an SM
+// are 16 and 128 results per clock.
 #pragma once
 
 #include "fa_common.cuh"
@@ -43,6 +51,7 @@ struct FwdParams {
     int N;
     int nqb;                  // query blocks of 128 rows
     int nkb;                  // key blocks of 128 keys
+    int nbh;                  // batch x heads
     int mode;                 // kCausal | kSparse bits
     float scale_log2;         // scale * log2(e)
 };
@@ -79,22 +88,22 @@ struct KvIter {
     }
 };
 
-template <int D, int NQ, int NS>
+template <int D, int NQ, int NSK, int NSV>
 struct FwdCfg {
     static constexpr int kChunks = D / 64;              // 128-byte swizzle atoms along d
     static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
     static constexpr int kTileBytes = 128 * D * 2;      // a 128-row tile of Q, K or V
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kQOff + NQ * kTileBytes;
-    static constexpr int kVOff = kKOff + NS * kTileBytes;
-    static constexpr int kBarOff = kVOff + NS * kTileBytes;
+    static constexpr int kVOff = kKOff + NSK * kTileBytes;
+    static constexpr int kBarOff = kVOff + NSV * kTileBytes;
     // barrier indices
     static constexpr int kBarQ = 0;
     static constexpr int kBarKFull = 1;
-    static constexpr int kBarVFull = kBarKFull + NS;
-    static constexpr int kBarKEmpty = kBarVFull + NS;
-    static constexpr int kBarVEmpty = kBarKEmpty + NS;
-    static constexpr int kBarSFull = kBarVEmpty + NS;
+    static constexpr int kBarVFull = kBarKFull + NSK;
+    static constexpr int kBarKEmpty = kBarVFull + NSV;
+    static constexpr int kBarVEmpty = kBarKEmpty + NSK;
+    static constexpr int kBarSFull = kBarVEmpty + NSV;
     static constexpr int kBarPFull = kBarSFull + NQ;
     static constexpr int kBarOFull = kBarPFull + NQ;
     static constexpr int kBarMmaDone = kBarOFull + NQ;
@@ -104,7 +113,16 @@ struct FwdCfg {
     static constexpr int kSoftmaxWarps = 4 * NQ;
     static constexpr int kWarpTma = kSoftmaxWarps;
     static constexpr int kWarpMma = kSoftmaxWarps + 1;
-    static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+    // NQ = 2: V tiles come from their own producer warp, so that K tiles (more
+    // stages, needed first) are never held up behind a V stage
+    static constexpr int kWarpTmaV = NQ == 2 ? kSoftmaxWarps + 2 : kWarpTma;
+    // NQ = 2: a third warpgroup (TMA, MMA, two idle warps) hands registers
+    // to the softmax warpgroups (setmaxnreg: 2 x 128 x 216 + 128 x 72 =
+    // 384 threads x 168 at launch).  NQ = 1: 6 warps, no reallocation.
+    static constexpr int kThreads = NQ == 2 ? 384 : 32 * (kSoftmaxWarps + 2);
+    static constexpr int kRegsSoftmax = 216;
+    static constexpr int kRegsCtl = 72;
+    static_assert(NQ == 1 || 2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= 384 * 168, "register split");
     static constexpr int kOCol = 256;
     static_assert(D == 64 || D == 128 || D == 256, "head dim");
     static_assert(256 + NQ * D <= 512, "TMEM columns");
@@ -126,21 +144,23 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int D, int NQ, int NS, bool BF16>
-__global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
+template <int D, int NQ, int NSK, int NSV, bool BF16>
+__global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
-    using C = FwdCfg<D, NQ, NS>;
+    using C = FwdCfg<D, NQ, NSK, NSV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
-    // causal: the heaviest query blocks start first
-    const int qp = (p.mode & kCausal) ? static_cast<int>(gridDim.y - 1 - blockIdx.y)
-                                      : static_cast<int>(blockIdx.y);
+    // one-dimensional grid, (batch, head) minor: causal runs the heaviest
+    // query blocks of every (b, h) first (longest work first balances the SMs)
+    const int nqp = (p.nqb + NQ - 1) / NQ;
+    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+    const int qi = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    const int qp = (p.mode & kCausal) ? nqp - 1 - qi : qi;
     const int rb0 = qp * NQ;
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
@@ -149,10 +169,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::kBarQ), 1);
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NSK; ++s) {
             mbar_init(bar(C::kBarKFull + s), 1);
-            mbar_init(bar(C::kBarVFull + s), 1);
             mbar_init(bar(C::kBarKEmpty + s), 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(bar(C::kBarVFull + s), 1);
             mbar_init(bar(C::kBarVEmpty + s), 1);
         }
         for (int t = 0; t < NQ; ++t) {
@@ -178,156 +200,167 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == C::kWarpTma) {
-        // ------------------------------------------------------------ producer
-        int nq_valid = 0;
-        for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
-            for (int t = 0; t < NQ; ++t) {
-                if (rb0 + t >= p.nqb) continue;
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
-                                bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
+    if (warp >= C::kSoftmaxWarps) {
+        if constexpr (NQ == 2) setmaxnreg_dec<C::kRegsCtl>();
+        if (warp == C::kWarpTma || warp == C::kWarpTmaV) {
+            // ------------------------------------------------------------ producer(s)
+            const bool do_k = warp == C::kWarpTma;
+            const bool do_v = warp == C::kWarpTmaV;
+            int nq_valid = 0;
+            for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
+            if (do_k && lane == 0) {
+                mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
+                for (int t = 0; t < NQ; ++t) {
+                    if (rb0 + t >= p.nqb) continue;
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
+                                    bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
+                }
             }
-        }
-        __syncwarp();
-        KvIter<NQ> it;
-        int j;
-        uint32_t f;
-        int nk = 0, nv = 0;   // loads issued
-        bool ok = true;
-        while (ok && it.next(p, rb0, j, f)) {
-            const int s = nk % NS;
-            const uint32_t ph = (nk / NS) & 1;
-            ok = wait_bar(bar(C::kBarKEmpty + s), ph ^ 1u, abort_flag);
-            if (!ok) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
-                                bar(C::kBarKFull + s), c * 64, j * 128, bh);
-            }
-            ++nk;
-            ok = wait_bar(bar(C::kBarVEmpty + s), ph ^ 1u, abort_flag);
-            if (!ok) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
-                                bar(C::kBarVFull + s), c * 64, j * 128, bh);
-            }
-            ++nv;
             __syncwarp();
-        }
-        // every issued load has landed before the CTA may exit
-        drain_bar(bar(C::kBarQ), 0);
-        for (int i = (nk > NS ? nk - NS : 0); i < nk; ++i)
-            drain_bar(bar(C::kBarKFull + i % NS), (i / NS) & 1);
-        for (int i = (nv > NS ? nv - NS : 0); i < nv; ++i)
-            drain_bar(bar(C::kBarVFull + i % NS), (i / NS) & 1);
-    } else if (warp == C::kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t kIdescS = instr_desc_f16(128, 128, BF16, false, false);
-        constexpr uint32_t kIdescO = instr_desc_f16(128, D, BF16, false, true);
-        // descriptors built once; each instruction only offsets the start address
-        const SmemDesc dQ = make_desc(sbase + C::kQOff, 16, 1024);
-        const SmemDesc dK = make_desc(sbase + C::kKOff, 16, 1024);
-        const SmemDesc dV = make_desc(sbase + C::kVOff, C::kChunkBytes, 1024);
-        auto issue_s = [&](int t, int s) {
-            const uint32_t d_tmem = tmem + 128u * t;
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const uint32_t koff = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
-                mma_ss(d_tmem, dQ.at(t * C::kTileBytes + koff), dK.at(s * C::kTileBytes + koff), kIdescS,
-                       k > 0 ? 1u : 0u);
-            }
-        };
-        auto issue_pv = [&](int t, int s, bool acc) {
-            const uint32_t d_tmem = tmem + C::kOCol + D * t;
-            const uint32_t a_tmem = tmem + 128u * t;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_ts(d_tmem, a_tmem + 8u * k, dV.at(s * C::kTileBytes + k * 2048), kIdescO,
-                       (acc || k > 0) ? 1u : 0u);
-        };
-
-        KvIter<NQ> it;
-        int j, jn;
-        uint32_t f, fn;
-        int cnt[NQ];
-#pragma unroll
-        for (int t = 0; t < NQ; ++t) cnt[t] = 0;
-        bool have = it.next(p, rb0, j, f);
-        bool ok = true;
-        if (have) {
-            ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                if (lane == 0) {
-                    for (int t = 0; t < NQ; ++t)
-                        if ((f >> t) & 1u) {
-                            issue_s(t, 0);
-                            mma_commit(bar(C::kBarSFull + t));
-                        }
-                    mma_commit(bar(C::kBarKEmpty));
+            KvIter<NQ> it;
+            int j;
+            uint32_t f;
+            int nk = 0, nv = 0;   // loads issued
+            bool ok = true;
+            while (ok && it.next(p, rb0, j, f)) {
+                if (do_k) {
+                    const int s = nk % NSK;
+                    ok = wait_bar(bar(C::kBarKEmpty + s), ((nk / NSK) & 1) ^ 1u, abort_flag);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
+                                        bar(C::kBarKFull + s), c * 64, j * 128, bh);
+                    }
+                    ++nk;
+                }
+                if (do_v) {
+                    const int s = nv % NSV;
+                    ok = wait_bar(bar(C::kBarVEmpty + s), ((nv / NSV) & 1) ^ 1u, abort_flag);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
+                                        bar(C::kBarVFull + s), c * 64, j * 128, bh);
+                    }
+                    ++nv;
                 }
                 __syncwarp();
             }
-        }
-        int u = 0;
-        while (ok && have) {
-            const int s = u % NS;
-            const uint32_t ph = (u / NS) & 1;
-            const bool have_n = it.next(p, rb0, jn, fn);
-            const int sn = (u + 1) % NS;
-            const uint32_t phn = ((u + 1) / NS) & 1;
-            ok = wait_bar(bar(C::kBarVFull + s), ph, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            bool k_ready = false;
+            // every issued load has landed before the CTA may exit
+            if (do_k) drain_bar(bar(C::kBarQ), 0);
+            for (int i = (nk > NSK ? nk - NSK : 0); i < nk; ++i)
+                drain_bar(bar(C::kBarKFull + i % NSK), (i / NSK) & 1);
+            for (int i = (nv > NSV ? nv - NSV : 0); i < nv; ++i)
+                drain_bar(bar(C::kBarVFull + i % NSV), (i / NSV) & 1);
+        } else if (warp == C::kWarpMma) {
+            // ------------------------------------------------------------ MMA issuer
+            const uint32_t leader = elect_one();   // the lane that issues tcgen05 ops
+            constexpr uint32_t kIdescS = instr_desc_f16(128, 128, BF16, false, false);
+            constexpr uint32_t kIdescO = instr_desc_f16(128, D, BF16, false, true);
+            // descriptors built once; each instruction only offsets the start address
+            const SmemDesc dQ = make_desc(sbase + C::kQOff, 16, 1024);
+            const SmemDesc dK = make_desc(sbase + C::kKOff, 16, 1024);
+            const SmemDesc dV = make_desc(sbase + C::kVOff, C::kChunkBytes, 1024);
+            auto issue_s = [&](int t, int s) {
+                const uint32_t d_tmem = tmem + 128u * t;
 #pragma unroll
-            for (int t = 0; t < NQ; ++t) {
-                if ((f >> t) & 1u) {
-                    ok = wait_bar(bar(C::kBarPFull + t), cnt[t] & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) issue_pv(t, s, cnt[t] > 0);
-                    __syncwarp();
-                    ++cnt[t];
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t koff = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
+                    mma_ss(d_tmem, dQ.at(t * C::kTileBytes + koff), dK.at(s * C::kTileBytes + koff), kIdescS,
+                           k > 0 ? 1u : 0u, leader);
                 }
-                if (have_n && ((fn >> t) & 1u)) {
-                    if (!k_ready) {
-                        ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
+            };
+            auto issue_pv = [&](int t, int s, bool acc) {
+                const uint32_t d_tmem = tmem + C::kOCol + D * t;
+                const uint32_t a_tmem = tmem + 128u * t;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(d_tmem, a_tmem + 8u * k, dV.at(s * C::kTileBytes + k * 2048), kIdescO,
+                           (acc || k > 0) ? 1u : 0u, leader);
+            };
+
+            KvIter<NQ> it;
+            int j, jn;
+            uint32_t f, fn;
+            int cnt[NQ];
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) cnt[t] = 0;
+            bool have = it.next(p, rb0, j, f);
+            bool ok = true;
+            if (have) {
+                ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    {
+                        for (int t = 0; t < NQ; ++t)
+                            if ((f >> t) & 1u) {
+                                issue_s(t, 0);
+                                mma_commit(bar(C::kBarSFull + t), leader);
+                            }
+                        mma_commit(bar(C::kBarKEmpty), leader);
+                    }
+                    __syncwarp();
+                }
+            }
+            int u = 0;
+            while (ok && have) {
+                const int s = u % NSV;                 // V stage of this key tile
+                const uint32_t ph = (u / NSV) & 1;
+                const bool have_n = it.next(p, rb0, jn, fn);
+                const int sn = (u + 1) % NSK;          // K stage of the next key tile
+                const uint32_t phn = ((u + 1) / NSK) & 1;
+                ok = wait_bar(bar(C::kBarVFull + s), ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                bool k_ready = false;
+#pragma unroll
+                for (int t = 0; t < NQ; ++t) {
+                    if ((f >> t) & 1u) {
+                        ok = wait_bar(bar(C::kBarPFull + t), cnt[t] & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        k_ready = true;
+                        issue_pv(t, s, cnt[t] > 0);
+                        __syncwarp();
+                        ++cnt[t];
                     }
-                    if (lane == 0) {
-                        issue_s(t, sn);
-                        mma_commit(bar(C::kBarSFull + t));
+                    if (have_n && ((fn >> t) & 1u)) {
+                        if (!k_ready) {
+                            ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        {
+                            issue_s(t, sn);
+                            mma_commit(bar(C::kBarSFull + t), leader);
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
+                if (!ok) break;
+                {
+                    mma_commit(bar(C::kBarVEmpty + s), leader);
+                    if (have_n) mma_commit(bar(C::kBarKEmpty + sn), leader);
+                }
+                __syncwarp();
+                j = jn;
+                f = fn;
+                have = have_n;
+                ++u;
             }
-            if (!ok) break;
-            if (lane == 0) {
-                mma_commit(bar(C::kBarVEmpty + s));
-                if (have_n) mma_commit(bar(C::kBarKEmpty + sn));
+            {
+                for (int t = 0; t < NQ; ++t) mma_commit(bar(C::kBarOFull + t), leader);
+                mma_commit(bar(C::kBarMmaDone), leader);
             }
             __syncwarp();
-            j = jn;
-            f = fn;
-            have = have_n;
-            ++u;
+            drain_bar(bar(C::kBarMmaDone), 0);
         }
-        if (lane == 0) {
-            for (int t = 0; t < NQ; ++t) mma_commit(bar(C::kBarOFull + t));
-            mma_commit(bar(C::kBarMmaDone));
-        }
-        __syncwarp();
-        drain_bar(bar(C::kBarMmaDone), 0);
     } else {
+        if constexpr (NQ == 2) setmaxnreg_inc<C::kRegsSoftmax>();
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int wq = warp & 3;
@@ -354,9 +387,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
             for (int q = 0; q < 4; ++q)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
             tmem_ld_wait();
-            float sv[128];
-#pragma unroll
-            for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
+            float *sv = reinterpret_cast<float *>(r);
             const bool diag = (p.mode & kCausal) && j == rb;
             const bool tail = (j == p.nkb - 1) && (p.N & 127);
             if (diag || tail) {
@@ -366,9 +397,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
                 for (int k = 0; k < 128; ++k)
                     if (k >= lim) sv[k] = -INFINITY;
             }
-            float mx = sv[0];
+            // row max: four independent chains of three-input max
+            float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
 #pragma unroll
-            for (int k = 1; k < 128; ++k) mx = fmaxf(mx, sv[k]);
+            for (int k = 4; k < 128; k += 8) {
+                mx0 = fmax3(mx0, sv[k], sv[k + 1]);
+                mx1 = fmax3(mx1, sv[k + 2], sv[k + 3]);
+                mx2 = fmax3(mx2, sv[k + 4], sv[k + 5]);
+                mx3 = fmax3(mx3, sv[k + 6], sv[k + 7]);
+            }
+            const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
             const float m_cand = fmaxf(m, mx * c);
             const bool grow = m_cand > m + 8.0f;    // lazy: keep m unless it moves by > 2^8
             const float m_new = grow ? m_cand : m;
@@ -386,24 +424,43 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NS>::kThreads, 1)
                     tmem_st32(tO + 32 * q, o);
                 }
             }
-            float sum = 0.f, sum_r = 0.f;
+            // P = 2^(s c - m): 3 of every 8 pairs on the FMA pipe (polynomial),
+            // the rest on the special-function unit
+            float2 acc[4], acc_r[4];
+#pragma unroll
+            for (int a4 = 0; a4 < 4; ++a4) acc[a4] = acc_r[a4] = make_float2(0.f, 0.f);
+            const float2 cc = make_float2(c, c), mm = make_float2(-m_use, -m_use);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const float p0 = ex2(fmaf(sv[32 * q + 2 * k], c, -m_use));
-                    const float p1 = ex2(fmaf(sv[32 * q + 2 * k + 1], c, -m_use));
-                    pk[k] = pack2<BF16>(p0, p1);
-                    sum += p0 + p1;
+                    const int g = 16 * q + k;
+                    const float2 x = ffma2(make_float2(sv[2 * g], sv[2 * g + 1]), cc, mm);
+                    float2 pr;
+                    if ((g & 7) >= 5) {
+                        pr = exp2_poly2(x);
+                    } else {
+                        pr.x = ex2(x.x);
+                        pr.y = ex2(x.y);
+                    }
+                    pk[k] = pack2<BF16>(pr.x, pr.y);
+                    acc[k & 3] = fadd2(acc[k & 3], pr);
                     if constexpr (BF16) {
                         // O is normalised by the sum of the same rounded P the
                         // tensor core multiplies (a row dominated by one key then
                         // comes out exact); LSE keeps the unrounded sum
-                        sum_r += __uint_as_float(pk[k] << 16) + __uint_as_float(pk[k] & 0xffff0000u);
+                        acc_r[k & 3] = fadd2(acc_r[k & 3], unpack2<true>(pk[k]));
                     }
                 }
                 tmem_st16(tS + 16 * q, pk);
+            }
+            const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+            const float sum = s01.x + s01.y;
+            float sum_r = 0.f;
+            if constexpr (BF16) {
+                const float2 r01 = fadd2(fadd2(acc_r[0], acc_r[1]), fadd2(acc_r[2], acc_r[3]));
+                sum_r = r01.x + r01.y;
             }
             l = l * alpha + sum;
             if constexpr (BF16) l_r = l_r * alpha + sum_r;

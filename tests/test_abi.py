@@ -58,7 +58,7 @@ def _fwd(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, scale=0.125, causal=0
     (dict(lse=NULL), INVALID),
     (dict(k=M), MISALIGNED),
     (dict(o=M), MISALIGNED),
-    (dict(N=300_000_000), UNSUPPORTED),   # more query-block pairs than a grid dimension holds
+    (dict(B=1 << 20, H=1 << 10, N=512), UNSUPPORTED),   # more CTAs than a one-dimensional grid holds
 ])
 def test_fwd_rejects(kw, expect):
     assert _fwd(**kw) == expect
