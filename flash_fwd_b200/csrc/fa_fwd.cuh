@@ -33,9 +33,10 @@
 //
 // Scale handling: exp is evaluated as 2^(s * scale * log2 e - m), with the
 // running max m kept in that base-2 domain; LSE converts back to natural log.
-// The exp2 work is split between the special-function unit and the FMA pipe
-// (a degree-3 polynomial for 3 of every 8 pairs), whose throughputs on an SM
-// are 16 and 128 results per clock.
+// exp2 runs on the special-function unit (16 results per clock per SM); a
+// degree-3 polynomial on the FMA pipe (128 per clock) can take a share of the
+// pairs (kPolyPairs), which measured slower here because the softmax warps
+// are issue-bound.
 #pragma once
 
 #include "fa_common.cuh"
@@ -424,8 +425,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     tmem_st32(tO + 32 * q, o);
                 }
             }
-            // P = 2^(s c - m): 3 of every 8 pairs on the FMA pipe (polynomial),
-            // the rest on the special-function unit
+            // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA pipe
+            // (polynomial) instead of the special-function unit; measured on
+            // B200 the softmax is issue-bound rather than MUFU-bound here, and
+            // moving any pairs made it slower, so all of them use MUFU.
+            constexpr int kPolyPairs = 0;
             float2 acc[4], acc_r[4];
 #pragma unroll
             for (int a4 = 0; a4 < 4; ++a4) acc[a4] = acc_r[a4] = make_float2(0.f, 0.f);
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     const int g = 16 * q + k;
                     const float2 x = ffma2(make_float2(sv[2 * g], sv[2 * g + 1]), cc, mm);
                     float2 pr;
-                    if ((g & 7) >= 5) {
+                    if ((g & 7) >= 8 - kPolyPairs) {
                         pr = exp2_poly2(x);
                     } else {
                         pr.x = ex2(x.x);
