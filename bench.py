@@ -97,7 +97,7 @@ def describe(name, w):
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "flash_fwd_b200", "csrc", "*"))):
+    for p in sorted(glob.glob(os.path.join(ROOT, "flash_fwd_b200", "csrc", "*.cu*"))):
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
