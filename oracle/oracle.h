@@ -17,6 +17,37 @@ extern "C" {
 
 #define ORACLE_CAUSAL 1
 #define ORACLE_SPARSE 2
+#define ORACLE_WINDOW 4   /* sliding window (left, right) */
+#define ORACLE_ALIBI 8    /* ALiBi bias -slope_h |i + Nk - Nq - j| */
+
+/*
+ * The _ex variants take Nq query rows and Nk keys per head (q, o, dout, dq:
+ * [BH][Nq][d]; k, v, dk, dv: [BH][Nk][d]; lse [BH][Nq]), bottom-right aligned
+ * (query i meets key i + Nk - Nq on the diagonal), a window (left, right)
+ * used with ORACLE_WINDOW (negative = unbounded side), ALiBi slopes [H]
+ * used with ORACLE_ALIBI (batch-head bh has head bh % H), and the block mask
+ * [ceil(Nq/blk)][ceil(Nk/blk)].  The plain variants are Nq = Nk = N, H = 1.
+ */
+int oracle_fwd_rows_ex(const double *q, const double *k, const double *v,
+                       int BH, int H, int Nq, int Nk, int d, double scale, int flags, int left, int right,
+                       const double *slopes, const uint8_t *mask, int blk, const int *rows, int nrows,
+                       double *o, double *lse, int nthreads);
+int oracle_online_softmax_fwd_ex(const double *q, const double *k, const double *v,
+                                 int Nq, int Nk, int d, double scale, int flags, int left, int right,
+                                 const double *slope, const uint8_t *mask, int blk, int tile,
+                                 double *o, double *lse);
+int oracle_bwd_full_ex(const double *q, const double *k, const double *v, const double *dout,
+                       int BH, int H, int Nq, int Nk, int d, double scale, int flags, int left, int right,
+                       const double *slopes, const uint8_t *mask, int blk,
+                       double *o, double *lse, double *dq, double *dk, double *dv, int nthreads);
+int oracle_bwd_dq_rows_ex(const double *q, const double *k, const double *v, const double *dout,
+                          int BH, int H, int Nq, int Nk, int d, double scale, int flags, int left, int right,
+                          const double *slopes, const uint8_t *mask, int blk, const int *rows, int nrows,
+                          double *dq, int nthreads);
+int oracle_bwd_dkdv_cols_ex(const double *q, const double *k, const double *v, const double *dout,
+                            int BH, int H, int Nq, int Nk, int d, double scale, int flags, int left, int right,
+                            const double *slopes, const uint8_t *mask, int blk, const int *cols, int ncols,
+                            double *dk, double *dv, int nthreads);
 
 /* O and LSE on the query rows listed in rows[nrows]; o is [BH][nrows][d], lse [BH][nrows] */
 int oracle_fwd_rows(const double *q, const double *k, const double *v,

@@ -5,8 +5,11 @@ CPU-baseline leg, never by the product package.
 
 Every function takes float64 numpy arrays laid out [BH, N, d] (one batch-head
 after another, the same order as the CUDA path's BHND tensors flattened over
-B and H) and returns float64 arrays.  The definitions computed are written out
-at the top of oracle.c with the passages they follow.
+B and H) and returns float64 arrays.  Queries and keys may differ in length:
+q and dout are [BH, Nq, d], k and v [BH, Nk, d] (bottom-right aligned).
+Optional modes: window=(left, right) (a negative side is unbounded) and
+slopes=[H] for ALiBi (batch-head bh uses slopes[bh % H]).  The definitions
+computed are written out at the top of oracle.c with the passages they follow.
 """
 import ctypes
 import os
@@ -16,6 +19,8 @@ import numpy as np
 
 CAUSAL = 1
 SPARSE = 2
+WINDOW = 4
+ALIBI = 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -48,13 +53,13 @@ def _lib():
         U8 = ctypes.POINTER(ctypes.c_uint8)
         I32 = ctypes.POINTER(ctypes.c_int)
         i, f = ctypes.c_int, ctypes.c_double
-        lib.oracle_fwd_rows.argtypes = [D, D, D, i, i, i, f, i, U8, i, I32, i, D, D, i]
-        lib.oracle_online_softmax_fwd.argtypes = [D, D, D, i, i, f, i, U8, i, i, D, D]
-        lib.oracle_bwd_full.argtypes = [D, D, D, D, i, i, i, f, i, U8, i, D, D, D, D, D, i]
-        lib.oracle_bwd_dq_rows.argtypes = [D, D, D, D, i, i, i, f, i, U8, i, I32, i, D, i]
-        lib.oracle_bwd_dkdv_cols.argtypes = [D, D, D, D, i, i, i, f, i, U8, i, I32, i, D, D, i]
-        for fn in (lib.oracle_fwd_rows, lib.oracle_online_softmax_fwd, lib.oracle_bwd_full,
-                   lib.oracle_bwd_dq_rows, lib.oracle_bwd_dkdv_cols):
+        lib.oracle_fwd_rows_ex.argtypes = [D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, I32, i, D, D, i]
+        lib.oracle_online_softmax_fwd_ex.argtypes = [D, D, D, i, i, i, f, i, i, i, D, U8, i, i, D, D]
+        lib.oracle_bwd_full_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, D, D, D, D, D, i]
+        lib.oracle_bwd_dq_rows_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, I32, i, D, i]
+        lib.oracle_bwd_dkdv_cols_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, I32, i, D, D, i]
+        for fn in (lib.oracle_fwd_rows_ex, lib.oracle_online_softmax_fwd_ex, lib.oracle_bwd_full_ex,
+                   lib.oracle_bwd_dq_rows_ex, lib.oracle_bwd_dkdv_cols_ex):
             fn.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -84,81 +89,116 @@ def _check_qkv(q, k, v):
     q, k, v = _f64(q), _f64(k), _f64(v)
     if q.ndim == 2:
         q, k, v = q[None], k[None], v[None]
-    assert q.shape == k.shape == v.shape and q.ndim == 3, "expected [BH, N, d]"
+    assert q.ndim == 3 and k.shape == v.shape and k.ndim == 3, "expected [BH, N, d]"
+    assert q.shape[0] == k.shape[0] and q.shape[2] == k.shape[2], "q [BH, Nq, d] and k, v [BH, Nk, d]"
     return q, k, v
 
 
-def fwd_rows(q, k, v, scale, flags=0, mask=None, blk=128, rows=None, nthreads=None):
+def _modes(flags, window, slopes):
+    """flags with WINDOW / ALIBI set from the arguments; (left, right, slopes array, H)."""
+    flags = int(flags)
+    left = right = -1
+    if window is not None:
+        flags |= WINDOW
+        left, right = int(window[0]), int(window[1])
+    sl = None
+    H = 1
+    if slopes is not None:
+        flags |= ALIBI
+        sl = np.ascontiguousarray(np.asarray(slopes, dtype=np.float64).reshape(-1))
+        H = len(sl)
+    return flags, left, right, sl, H
+
+
+def _sp(a):
+    return None if a is None else _dp(a)
+
+
+def fwd_rows(q, k, v, scale, flags=0, mask=None, blk=128, rows=None, nthreads=None, window=None, slopes=None):
     """O [BH, len(rows), d] and LSE [BH, len(rows)] on the given query rows."""
     q, k, v = _check_qkv(q, k, v)
-    BH, N, d = q.shape
-    rows = np.arange(N, dtype=np.int32) if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    BH, Nq, d = q.shape
+    Nk = k.shape[1]
+    fl, left, right, sl, H = _modes(flags, window, slopes)
+    rows = np.arange(Nq, dtype=np.int32) if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
     o = np.zeros((BH, len(rows), d))
     lse = np.zeros((BH, len(rows)))
     m, mp = _mask_arg(mask)
-    rc = _lib().oracle_fwd_rows(_dp(q), _dp(k), _dp(v), BH, N, d, float(scale), int(flags), mp, int(blk),
-                                rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(rows),
-                                _dp(o), _dp(lse), _threads(nthreads))
+    rc = _lib().oracle_fwd_rows_ex(_dp(q), _dp(k), _dp(v), BH, H, Nq, Nk, d, float(scale), fl, left, right,
+                                   _sp(sl), mp, int(blk), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                   len(rows), _dp(o), _dp(lse), _threads(nthreads))
     assert rc == 0, rc
     return o, lse
 
 
-def fwd(q, k, v, scale, flags=0, mask=None, blk=128, nthreads=None):
+def fwd(q, k, v, scale, flags=0, mask=None, blk=128, nthreads=None, window=None, slopes=None):
     """O and LSE on every query row."""
-    return fwd_rows(q, k, v, scale, flags, mask, blk, None, nthreads)
+    return fwd_rows(q, k, v, scale, flags, mask, blk, None, nthreads, window, slopes)
 
 
-def online_softmax_fwd(q, k, v, scale, tile, flags=0, mask=None, blk=128):
-    """One head [N, d]: the tiled online-softmax recurrence with `tile` keys per step."""
+def online_softmax_fwd(q, k, v, scale, tile, flags=0, mask=None, blk=128, window=None, slope=None):
+    """One head (q [Nq, d], k, v [Nk, d]): the tiled online-softmax recurrence with `tile` keys per step."""
     q, k, v = _f64(q), _f64(k), _f64(v)
-    N, d = q.shape
-    o = np.zeros((N, d))
-    lse = np.zeros(N)
+    Nq, d = q.shape
+    Nk = k.shape[0]
+    fl, left, right, sl, _ = _modes(flags, window, None if slope is None else [slope])
+    o = np.zeros((Nq, d))
+    lse = np.zeros(Nq)
     m, mp = _mask_arg(mask)
-    rc = _lib().oracle_online_softmax_fwd(_dp(q), _dp(k), _dp(v), N, d, float(scale), int(flags), mp,
-                                          int(blk), int(tile), _dp(o), _dp(lse))
+    rc = _lib().oracle_online_softmax_fwd_ex(_dp(q), _dp(k), _dp(v), Nq, Nk, d, float(scale), fl, left, right,
+                                             _sp(sl), mp, int(blk), int(tile), _dp(o), _dp(lse))
     assert rc == 0, rc
     return o, lse
 
 
-def bwd_full(q, k, v, dout, scale, flags=0, mask=None, blk=128, nthreads=None):
-    """(O, LSE, dQ, dK, dV), materialising the N x N matrices of every head."""
+def bwd_full(q, k, v, dout, scale, flags=0, mask=None, blk=128, nthreads=None, window=None, slopes=None):
+    """(O, LSE, dQ, dK, dV), materialising the Nq x Nk matrices of every head."""
     q, k, v = _check_qkv(q, k, v)
     dout = _f64(dout).reshape(q.shape)
-    BH, N, d = q.shape
-    o, dq, dk, dv = (np.zeros_like(q) for _ in range(4))
-    lse = np.zeros((BH, N))
+    BH, Nq, d = q.shape
+    Nk = k.shape[1]
+    fl, left, right, sl, H = _modes(flags, window, slopes)
+    o, dq = np.zeros_like(q), np.zeros_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(k)
+    lse = np.zeros((BH, Nq))
     m, mp = _mask_arg(mask)
-    rc = _lib().oracle_bwd_full(_dp(q), _dp(k), _dp(v), _dp(dout), BH, N, d, float(scale), int(flags), mp,
-                                int(blk), _dp(o), _dp(lse), _dp(dq), _dp(dk), _dp(dv), _threads(nthreads))
+    rc = _lib().oracle_bwd_full_ex(_dp(q), _dp(k), _dp(v), _dp(dout), BH, H, Nq, Nk, d, float(scale), fl, left,
+                                   right, _sp(sl), mp, int(blk), _dp(o), _dp(lse), _dp(dq), _dp(dk), _dp(dv),
+                                   _threads(nthreads))
     assert rc == 0, rc
     return o, lse, dq, dk, dv
 
 
-def bwd_dq_rows(q, k, v, dout, scale, rows, flags=0, mask=None, blk=128, nthreads=None):
+def bwd_dq_rows(q, k, v, dout, scale, rows, flags=0, mask=None, blk=128, nthreads=None, window=None, slopes=None):
     q, k, v = _check_qkv(q, k, v)
     dout = _f64(dout).reshape(q.shape)
-    BH, N, d = q.shape
+    BH, Nq, d = q.shape
+    Nk = k.shape[1]
+    fl, left, right, sl, H = _modes(flags, window, slopes)
     rows = np.ascontiguousarray(rows, dtype=np.int32)
     dq = np.zeros((BH, len(rows), d))
     m, mp = _mask_arg(mask)
-    rc = _lib().oracle_bwd_dq_rows(_dp(q), _dp(k), _dp(v), _dp(dout), BH, N, d, float(scale), int(flags), mp,
-                                   int(blk), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(rows),
-                                   _dp(dq), _threads(nthreads))
+    rc = _lib().oracle_bwd_dq_rows_ex(_dp(q), _dp(k), _dp(v), _dp(dout), BH, H, Nq, Nk, d, float(scale), fl, left,
+                                      right, _sp(sl), mp, int(blk), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                      len(rows), _dp(dq), _threads(nthreads))
     assert rc == 0, rc
     return dq
 
 
-def bwd_dkdv_cols(q, k, v, dout, scale, cols, flags=0, mask=None, blk=128, nthreads=None):
+def bwd_dkdv_cols(q, k, v, dout, scale, cols, flags=0, mask=None, blk=128, nthreads=None, window=None,
+                  slopes=None):
     q, k, v = _check_qkv(q, k, v)
     dout = _f64(dout).reshape(q.shape)
-    BH, N, d = q.shape
+    BH, Nq, d = q.shape
+    Nk = k.shape[1]
+    fl, left, right, sl, H = _modes(flags, window, slopes)
     cols = np.ascontiguousarray(cols, dtype=np.int32)
     dk = np.zeros((BH, len(cols), d))
     dv = np.zeros((BH, len(cols), d))
     m, mp = _mask_arg(mask)
-    rc = _lib().oracle_bwd_dkdv_cols(_dp(q), _dp(k), _dp(v), _dp(dout), BH, N, d, float(scale), int(flags), mp,
-                                     int(blk), cols.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(cols),
-                                     _dp(dk), _dp(dv), _threads(nthreads))
+    rc = _lib().oracle_bwd_dkdv_cols_ex(_dp(q), _dp(k), _dp(v), _dp(dout), BH, H, Nq, Nk, d, float(scale), fl,
+                                        left, right, _sp(sl), mp, int(blk),
+                                        cols.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(cols),
+                                        _dp(dk), _dp(dv), _threads(nthreads))
     assert rc == 0, rc
     return dk, dv

@@ -17,17 +17,25 @@ SRC = os.path.join(ROOT, "oracle", "oracle.c")
 
 MUTANTS = {
     "dk_scale_dropped": ("dk[(size_t)j * d + x] = c->scale * acc;", "dk[(size_t)j * d + x] = acc;"),
-    "ds_sign_flipped": ("(dP[(size_t)i * N + j] - D[i])", "(D[i] - dP[(size_t)i * N + j])"),
-    "causal_off_by_one": ("if ((flags & ORACLE_CAUSAL) && j > i) return 0;",
-                          "if ((flags & ORACLE_CAUSAL) && j >= i) return 0;"),
-    "dv_operand_transposed": ("acc += P[(size_t)i * N + j] * dout[(size_t)i * d + x];",
-                              "acc += P[(size_t)j * N + i] * dout[(size_t)i * d + x];"),
+    "ds_sign_flipped": ("(dP[(size_t)i * Nk + j] - D[i])", "(D[i] - dP[(size_t)i * Nk + j])"),
+    "causal_off_by_one": ("if ((sp->flags & ORACLE_CAUSAL) && j > i + off) return 0;",
+                          "if ((sp->flags & ORACLE_CAUSAL) && j >= i + off) return 0;"),
+    "dv_operand_transposed": ("acc += P[(size_t)i * Nk + j] * dout[(size_t)i * d + x];",
+                              "acc += P[(size_t)j * Nk + i] * dout[(size_t)i * d + x];"),
     "lse_max_dropped": ("double lse = m + log(l);", "double lse = log(l);"),
-    "mask_index_transposed": ("!mask[(size_t)(i / blk) * nbk + (j / blk)]",
-                              "!mask[(size_t)(j / blk) * nbk + (i / blk)]"),
-    "scale_dropped_in_scores": ("srow[j] = scale * acc;", "srow[j] = acc;"),
+    "mask_index_transposed": ("!sp->mask[(size_t)(i / sp->blk) * sp->nbk + (j / sp->blk)]",
+                              "!sp->mask[(size_t)(j / sp->blk) * sp->nbk + (i / sp->blk)]"),
+    "scale_dropped_in_scores": ("srow[j] = scale * acc + bias(sp, h, i, j);", "srow[j] = acc + bias(sp, h, i, j);"),
+    # extended modes (Nq != Nk, sliding window, ALiBi)
+    "alignment_offset_dropped": ("const long off = (long)sp->Nk - sp->Nq;", "const long off = 0;"),
+    "window_left_off_by_one": ("if (sp->left >= 0 && j < i + off - sp->left) return 0;",
+                               "if (sp->left >= 0 && j <= i + off - sp->left) return 0;"),
+    "window_right_ignored": ("if (sp->right >= 0 && j > i + off + sp->right) return 0;", ""),
+    "alibi_sign_flipped": ("return -sp->slopes[h % sp->H] * dist;", "return sp->slopes[h % sp->H] * dist;"),
+    "alibi_offset_dropped": ("const double dist = fabs((double)i + ((double)sp->Nk - sp->Nq) - (double)j);",
+                             "const double dist = fabs((double)i - (double)j);"),
+    "alibi_head_ignored": ("return -sp->slopes[h % sp->H] * dist;", "return -sp->slopes[0] * dist;"),
 }
-
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
@@ -42,6 +50,7 @@ def test_pins_catch_mutant(name, tmp_path):
                     "-o", str(lib), str(cfile), "-lm", "-lpthread"], check=True)
     env = dict(os.environ, ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_modes.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
