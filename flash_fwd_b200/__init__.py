@@ -15,6 +15,7 @@ __all__ = [
     "FaError", "load_library", "library_path", "fa_fwd", "fa_fwd_blocksparse", "fa_bwd",
     "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status", "fa_last_timeout_site",
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
+    "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes",
 ]
 
 FA_BLOCK = 128
@@ -51,6 +52,10 @@ def load_library():
     lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, i, vp]
     lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, vp, i, vp]
+    lib.fa_bwd_ex_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_ex_workspace_bytes.restype = sz
+    lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, i, vp, vp, i, vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -58,7 +63,7 @@ def load_library():
     lib.fa_last_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
-    for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse,
+    for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -171,12 +176,53 @@ def fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask,
     _check(rc, "fa_bwd_blocksparse")
 
 
-def attention_fwd(q, k, v, causal=False, scale=None, block_mask=None, stream=None):
-    """Allocates O and LSE with torch and runs the forward; returns (o, lse)."""
-    B, H, N, d = _shape(q)
+def _window(window):
+    return (-1, -1) if window is None else (int(window[0]), int(window[1]))
+
+
+def fa_fwd_ex(q, k, v, o, lse, causal=False, scale=None, window=None, alibi_slopes=None, block_mask=None,
+              stream=None):
+    """General forward: q, o [B, H, Nq, d]; k, v [B, H, Nk, d]; lse [B, H, Nq] fp32.
+    window=(left, right) (a negative side is unbounded), alibi_slopes: fp32 [H] on the device."""
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
+    wl, wr = _window(window)
+    rc = load_library().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                  _scale(scale, d), int(bool(causal)), wl, wr, _ptr(alibi_slopes), _ptr(block_mask),
+                                  _dtype(q), _stream(stream))
+    _check(rc, "fa_fwd_ex")
+
+
+def fa_bwd_ex_workspace_bytes(B, H, Nq, Nk, d):
+    return load_library().fa_bwd_ex_workspace_bytes(B, H, Nq, Nk, d)
+
+
+def fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, window=None,
+              alibi_slopes=None, block_mask=None, stream=None):
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
+    wl, wr = _window(window)
+    rc = load_library().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)), wl, wr, _ptr(alibi_slopes),
+                                  _ptr(block_mask), _dtype(q), _stream(stream))
+    _check(rc, "fa_bwd_ex")
+
+
+def _general(q, k, window, alibi_slopes):
+    return k.shape[2] != q.shape[2] or window is not None or alibi_slopes is not None
+
+
+def attention_fwd(q, k, v, causal=False, scale=None, block_mask=None, stream=None, window=None,
+                  alibi_slopes=None):
+    """Allocates O and LSE with torch and runs the forward; returns (o, lse).
+    k, v may have a different length from q (bottom-right aligned)."""
+    B, H, Nq, d = _shape(q)
     o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if block_mask is None:
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if _general(q, k, window, alibi_slopes):
+        fa_fwd_ex(q, k, v, o, lse, causal, scale, window, alibi_slopes, block_mask, stream)
+    elif block_mask is None:
         fa_fwd(q, k, v, o, lse, causal, scale, stream)
     else:
         fa_fwd_blocksparse(q, k, v, o, lse, block_mask, causal, scale, stream)
@@ -184,13 +230,17 @@ def attention_fwd(q, k, v, causal=False, scale=None, block_mask=None, stream=Non
 
 
 def attention_bwd(q, k, v, o, dout, lse, causal=False, scale=None, block_mask=None, workspace=None,
-                  stream=None):
+                  stream=None, window=None, alibi_slopes=None):
     """Allocates dQ, dK, dV (and the workspace unless given) and runs the backward."""
-    B, H, N, d = _shape(q)
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
-    if block_mask is None:
+        workspace = torch.empty(fa_bwd_ex_workspace_bytes(B, H, Nq, Nk, d), dtype=torch.uint8, device=q.device)
+    if _general(q, k, window, alibi_slopes):
+        fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal, scale, window, alibi_slopes, block_mask,
+                  stream)
+    elif block_mask is None:
         fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal, scale, stream)
     else:
         fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask, causal, scale, stream)

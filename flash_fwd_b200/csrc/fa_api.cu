@@ -84,21 +84,46 @@ int make_map(CUtensorMap *map, const void *base, int d, int N, long long BH, int
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-int check_common(int B, int H, int N, int d, float scale, int dtype) {
-    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
-    if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-    const long long BH = static_cast<long long>(B) * H;
-    if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+// One attention problem as the entry points describe it.  Window sides and
+// ALiBi are optional (negative side = unbounded, null slopes = no bias).
+struct Problem {
+    int B, H, Nq, Nk, d;
+    float scale;
+    int causal;
+    int win_left, win_right;
+    const float *alibi;        // DEVICE [H]
+    const uint8_t *mask;       // DEVICE [ceil(Nq/128)][ceil(Nk/128)]
+    int dtype;
+    long long BH() const { return static_cast<long long>(B) * H; }
+    int off() const { return Nk - Nq; }
+    int wl() const { return win_left < 0 ? fa::kUnbounded : (win_left < fa::kUnbounded ? win_left : fa::kUnbounded); }
+    int wr() const {   // causal caps the right side at the diagonal
+        if (causal) return 0;
+        return win_right < 0 ? fa::kUnbounded : (win_right < fa::kUnbounded ? win_right : fa::kUnbounded);
+    }
+    int mode() const { return (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0); }
+};
+
+Problem square(int B, int H, int N, int d, float scale, int causal, const uint8_t *mask, int dtype) {
+    return Problem{B, H, N, N, d, scale, causal, -1, -1, nullptr, mask, dtype};
+}
+
+int check_problem(const Problem &pr) {
+    if (pr.B < 1 || pr.H < 1 || pr.Nq < 1 || pr.Nk < 1) return FA_ERR_INVALID_ARG;
+    if (pr.Nq > fa::kMaxRows || pr.Nk > fa::kMaxRows) return FA_ERR_UNSUPPORTED;
+    if (pr.dtype != FA_F16 && pr.dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(pr.scale) || !(pr.scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (pr.d != 64 && pr.d != 128 && pr.d != 256) return FA_ERR_UNSUPPORTED;
+    if (pr.BH() > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    if (pr.alibi && (reinterpret_cast<uintptr_t>(pr.alibi) & 3u)) return FA_ERR_MISALIGNED;
     return FA_OK;
 }
 
-template <int D, int NQ, int NSK, int NSV, bool BF16>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool ALIBI>
 int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const fa::FwdParams &p,
                int BH, cudaStream_t stream) {
     using C = fa::FwdCfg<D, NQ, NSK, NSV>;
-    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16>;
+    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, ALIBI>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     const long long ctas = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
@@ -109,43 +134,52 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <bool BF16>
+template <bool BF16, bool ALIBI>
 int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                  const fa::FwdParams &p, int BH, cudaStream_t s) {
     switch (d) {
-        case 64: return launch_fwd<64, 2, 6, 4, BF16>(mq, mk, mv, p, BH, s);
-        case 128: return launch_fwd<128, 2, 3, 2, BF16>(mq, mk, mv, p, BH, s);
-        case 256: return launch_fwd<256, 1, 1, 1, BF16>(mq, mk, mv, p, BH, s);
+        case 64: return launch_fwd<64, 2, 6, 4, BF16, ALIBI>(mq, mk, mv, p, BH, s);
+        case 128: return launch_fwd<128, 2, 3, 2, BF16, ALIBI>(mq, mk, mv, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, 1, BF16, ALIBI>(mq, mk, mv, p, BH, s);
         default: return FA_ERR_UNSUPPORTED;
     }
 }
 
-int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, const uint8_t *mask, int B,
-             int H, int N, int d, float scale, int causal, int dtype, void *stream) {
+int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, const Problem &pr, void *stream) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    int rc = check_common(B, H, N, d, scale, dtype);
+    int rc = check_problem(pr);
     if (rc != FA_OK) return rc;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_MISALIGNED;
-    const int BH = B * H;
-    if (static_cast<long long>(BH) * ((N + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // 1-D grid
+    const int BH = static_cast<int>(pr.BH());
+    if (static_cast<long long>(BH) * ((pr.Nq + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // 1-D grid
     CUtensorMap mq, mk, mv;
-    if ((rc = make_map(&mq, q, d, N, BH, dtype, 128)) != FA_OK) return rc;
-    if ((rc = make_map(&mk, k, d, N, BH, dtype, 128)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, d, N, BH, dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, q, pr.d, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, k, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, v, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     fa::FwdParams p;
     p.o = o;
     p.lse = lse;
-    p.mask = mask;
-    p.N = N;
-    p.nqb = (N + 127) / 128;
-    p.nkb = p.nqb;
+    p.mask = pr.mask;
+    p.alibi = pr.alibi;
+    p.Nq = pr.Nq;
+    p.Nk = pr.Nk;
+    p.off = pr.off();
+    p.wl = pr.wl();
+    p.wr = pr.wr();
+    p.nqb = (pr.Nq + 127) / 128;
+    p.nkb = (pr.Nk + 127) / 128;
     p.nbh = BH;
-    p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
-    p.scale_log2 = scale * kLog2e;
+    p.H = pr.H;
+    p.mode = pr.mode();
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * kLog2e;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return dtype == FA_BF16 ? dispatch_fwd<true>(d, mq, mk, mv, p, BH, s)
-                            : dispatch_fwd<false>(d, mq, mk, mv, p, BH, s);
+    if (pr.dtype == FA_BF16)
+        return pr.alibi ? dispatch_fwd<true, true>(pr.d, mq, mk, mv, p, BH, s)
+                        : dispatch_fwd<true, false>(pr.d, mq, mk, mv, p, BH, s);
+    return pr.alibi ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, p, BH, s)
+                    : dispatch_fwd<false, false>(pr.d, mq, mk, mv, p, BH, s);
 }
 
 
@@ -174,100 +208,100 @@ int launch_bwd_post(const float *dqacc, void *dq, long long elems, float scale, 
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+struct BwdBuffers {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv, *workspace;
+};
+
 // Three launches: pre-pass, main kernel (Kernel: a bwd_kernel or bwd_split_kernel
-// instantiation, BM query rows per tile, grid from MakeGrid), post-pass.
-template <int D, int BM, bool BF16, typename Kernel, typename MakeGrid>
-int launch_bwd(Kernel kern, int smem_bytes, int threads, MakeGrid make_grid, const void *q, const void *k,
-               const void *v, const void *o, const void *dout, const float *lse, void *dq, void *dk, void *dv,
-               void *workspace, const uint8_t *mask, int BH, int N, float scale, int causal, int dtype,
+// instantiation, BM query rows per tile, `split` CTAs per key block), post-pass.
+template <int D, int BM, bool BF16, typename Kernel>
+int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuffers &bb, const Problem &pr,
                cudaStream_t stream) {
-    const int Npad = fa::bwd_npad(N);
-    float *lse2 = static_cast<float *>(workspace);
+    const int BH = static_cast<int>(pr.BH());
+    const int Npad = fa::bwd_npad(pr.Nq);
+    float *lse2 = static_cast<float *>(bb.workspace);
     float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
     float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
-    int rc = launch_bwd_pre<D, BF16>(o, dout, lse, lse2, dvec, dqacc, BH, N, Npad, stream);
+    int rc = launch_bwd_pre<D, BF16>(bb.o, bb.dout, bb.lse, lse2, dvec, dqacc, BH, pr.Nq, Npad, stream);
     if (rc != FA_OK) return rc;
     CUtensorMap mk, mv, mq, mdo;
-    if ((rc = make_map(&mk, k, D, N, BH, dtype, 128)) != FA_OK) return rc;
-    if ((rc = make_map(&mv, v, D, N, BH, dtype, 128)) != FA_OK) return rc;
-    if ((rc = make_map(&mq, q, D, N, BH, dtype, BM)) != FA_OK) return rc;
-    if ((rc = make_map(&mdo, dout, D, N, BH, dtype, BM)) != FA_OK) return rc;
+    if ((rc = make_map(&mk, bb.k, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mv, bb.v, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mq, bb.q, D, pr.Nq, BH, pr.dtype, BM)) != FA_OK) return rc;
+    if ((rc = make_map(&mdo, bb.dout, D, pr.Nq, BH, pr.dtype, BM)) != FA_OK) return rc;
     fa::BwdParams p;
     p.lse2 = lse2;
     p.dvec = dvec;
     p.dqacc = dqacc;
-    p.dk = dk;
-    p.dv = dv;
-    p.mask = mask;
-    p.N = N;
+    p.dk = bb.dk;
+    p.dv = bb.dv;
+    p.mask = pr.mask;
+    p.alibi = pr.alibi;
+    p.Nq = pr.Nq;
+    p.Nk = pr.Nk;
+    p.off = pr.off();
+    p.wl = pr.wl();
+    p.wr = pr.wr();
+    p.H = pr.H;
     p.Npad = Npad;
-    p.nkb = (N + 127) / 128;
-    p.nqt = (N + BM - 1) / BM;
+    p.nkb = (pr.Nk + 127) / 128;
+    p.nqt = (pr.Nq + BM - 1) / BM;
     p.nbh = BH;
-    p.mode = (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0);
-    p.scale = scale;
-    p.scale_log2 = scale * kLog2e;
+    p.mode = pr.mode();
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * kLog2e;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
         return FA_ERR_CUDA;
     {
+        // one-dimensional grid of BH x key blocks (x split) CTAs
+        const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb * split));
         ProfScope prof(2, stream);
-        kern<<<make_grid(p.nkb, BH), threads, smem_bytes, stream>>>(mk, mv, mq, mdo, p);
+        kern<<<grid, threads, smem_bytes, stream>>>(mk, mv, mq, mdo, p);
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    return launch_bwd_post<BF16>(dqacc, dq, static_cast<long long>(BH) * N * D, scale, stream);
+    return launch_bwd_post<BF16>(dqacc, bb.dq, static_cast<long long>(BH) * pr.Nq * D, pr.scale, stream);
 }
 
-template <bool BF16>
-int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *o, const void *dout,
-                 const float *lse, void *dq, void *dk, void *dv, void *ws, const uint8_t *mask,
-                 int BH, int N, float scale, int causal, int dtype, cudaStream_t s) {
-    // One-dimensional grids of BH x key blocks CTAs (x 2 at d = 256: two CTAs
-    // per key block).
-    auto grid_bh_j = [](int nkb, int bh) { return dim3(static_cast<unsigned>(static_cast<long long>(bh) * nkb)); };
-    auto grid_split = [](int nkb, int bh) { return dim3(static_cast<unsigned>(static_cast<long long>(bh) * nkb * 2)); };
-    switch (d) {
+template <bool BF16, bool ALIBI>
+int dispatch_bwd(const BwdBuffers &bb, const Problem &pr, cudaStream_t s) {
+    switch (pr.d) {
         case 64: {
             using C = fa::BwdCfg<64, 3>;
-            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16>, C::kSmemBytes, C::kThreads, grid_bh_j,
-                                             q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH, N, scale, causal,
-                                             dtype, s);
+            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16, ALIBI>, C::kSmemBytes, C::kThreads, 1, bb,
+                                             pr, s);
         }
         case 128: {
             using C = fa::BwdCfg<128, 2>;
-            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16>, C::kSmemBytes, C::kThreads, grid_bh_j,
-                                              q, k, v, o, dout, lse, dq, dk, dv, ws, mask, BH, N, scale, causal,
-                                              dtype, s);
+            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16, ALIBI>, C::kSmemBytes, C::kThreads, 1,
+                                              bb, pr, s);
         }
         case 256: {
             using C = fa::BwdSplitCfg<256, 64, 2, 1, 2, true>;
-            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16>, C::kSmemBytes,
-                                             C::kThreads, grid_split, q, k, v, o, dout, lse, dq, dk, dv, ws, mask,
-                                             BH, N, scale, causal, dtype, s);
+            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, ALIBI>,
+                                             C::kSmemBytes, C::kThreads, 2, bb, pr, s);
         }
         default: return FA_ERR_UNSUPPORTED;
     }
 }
 
-int bwd_impl(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
-             void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, const uint8_t *mask, int B,
-             int H, int N, int d, float scale, int causal, int dtype, void *stream) {
-    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-    int rc = check_common(B, H, N, d, scale, dtype);
+int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, void *stream) {
+    if (!bb.q || !bb.k || !bb.v || !bb.o || !bb.dout || !bb.lse || !bb.dq || !bb.dk || !bb.dv)
+        return FA_ERR_INVALID_ARG;
+    int rc = check_problem(pr);
     if (rc != FA_OK) return rc;
-    const void *ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
+    const void *ptrs[] = {bb.q, bb.k, bb.v, bb.o, bb.dout, bb.lse, bb.dq, bb.dk, bb.dv};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
-    const long long BH = static_cast<long long>(B) * H;
-    if (BH * (2LL * ((N + 127) / 128)) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
-    const size_t need = fa::bwd_workspace_bytes(BH, N, d);
-    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+    if (pr.BH() * (2LL * ((pr.Nk + 127) / 128)) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
+    const size_t need = fa::bwd_workspace_bytes(pr.BH(), pr.Nq, pr.d);
+    if (!bb.workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (!aligned16(bb.workspace)) return FA_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return dtype == FA_BF16
-               ? dispatch_bwd<true>(d, q, k, v, o, dout, lse, dq, dk, dv, workspace, mask, static_cast<int>(BH), N,
-                                    scale, causal, dtype, s)
-               : dispatch_bwd<false>(d, q, k, v, o, dout, lse, dq, dk, dv, workspace, mask, static_cast<int>(BH),
-                                     N, scale, causal, dtype, s);
+    if (pr.dtype == FA_BF16)
+        return pr.alibi ? dispatch_bwd<true, true>(bb, pr, s) : dispatch_bwd<true, false>(bb, pr, s);
+    return pr.alibi ? dispatch_bwd<false, true>(bb, pr, s) : dispatch_bwd<false, false>(bb, pr, s);
 }
 
 // ---------------------------------------------------------------- fa_bwd_noalloc
@@ -301,14 +335,21 @@ extern "C" {
 
 FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
                   float scale, int causal, int dtype, void *stream) {
-    return fwd_impl(q, k, v, o, lse, nullptr, B, H, N, d, scale, causal, dtype, stream);
+    return fwd_impl(q, k, v, o, lse, square(B, H, N, d, scale, causal, nullptr, dtype), stream);
 }
 
 FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
                               const uint8_t *block_mask, int B, int H, int N, int d, float scale, int causal,
                               int dtype, void *stream) {
     if (!block_mask) return FA_ERR_INVALID_ARG;
-    return fwd_impl(q, k, v, o, lse, block_mask, B, H, N, d, scale, causal, dtype, stream);
+    return fwd_impl(q, k, v, o, lse, square(B, H, N, d, scale, causal, block_mask, dtype), stream);
+}
+
+FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int Nq,
+                     int Nk, int d, float scale, int causal, int window_left, int window_right,
+                     const float *alibi_slopes, const uint8_t *block_mask, int dtype, void *stream) {
+    const Problem pr{B, H, Nq, Nk, d, scale, causal, window_left, window_right, alibi_slopes, block_mask, dtype};
+    return fwd_impl(q, k, v, o, lse, pr, stream);
 }
 
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -316,11 +357,16 @@ FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
     return fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d);
 }
 
+FA_API size_t fa_bwd_ex_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
+    if (Nk < 1) return 0;
+    return fa_bwd_workspace_bytes(B, H, Nq, d);
+}
+
 FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
                   void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int N,
                   int d, float scale, int causal, int dtype, void *stream) {
-    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, nullptr, B, H, N, d, scale,
-                    causal, dtype, stream);
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    return bwd_impl(bb, workspace_bytes, square(B, H, N, d, scale, causal, nullptr, dtype), stream);
 }
 
 FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const void *dout,
@@ -328,21 +374,32 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
                               size_t workspace_bytes, const uint8_t *block_mask, int B, int H, int N, int d,
                               float scale, int causal, int dtype, void *stream) {
     if (!block_mask) return FA_ERR_INVALID_ARG;
-    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, block_mask, B, H, N, d, scale,
-                    causal, dtype, stream);
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    return bwd_impl(bb, workspace_bytes, square(B, H, N, d, scale, causal, block_mask, dtype), stream);
+}
+
+FA_API int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                     const float *lse, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                     int B, int H, int Nq, int Nk, int d, float scale, int causal, int window_left,
+                     int window_right, const float *alibi_slopes, const uint8_t *block_mask, int dtype,
+                     void *stream) {
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    const Problem pr{B, H, Nq, Nk, d, scale, causal, window_left, window_right, alibi_slopes, block_mask, dtype};
+    return bwd_impl(bb, workspace_bytes, pr, stream);
 }
 
 FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,
                           const float *lse, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
                           int causal, int dtype, void *stream) {
-    int rc = check_common(B, H, N, d, scale, dtype);
+    const Problem pr = square(B, H, N, d, scale, causal, nullptr, dtype);
+    int rc = check_problem(pr);
     if (rc != FA_OK) return rc;
-    const size_t need = fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d);
+    const size_t need = fa::bwd_workspace_bytes(pr.BH(), N, d);
     if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
     if ((rc = noalloc_scratch(&scratch)) != FA_OK) return rc;
-    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, nullptr, B, H, N, d,
-                    scale, causal, dtype, stream);
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, scratch};
+    return bwd_impl(bb, FA_NOALLOC_SCRATCH_BYTES, pr, stream);
 }
 
 FA_API const char *fa_status_string(int status) {

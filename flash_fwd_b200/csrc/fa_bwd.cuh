@@ -36,14 +36,17 @@
 namespace fa {
 
 struct BwdParams {
-    const float *lse2;    // [BH][Npad] LSE * log2(e) (+inf for rows past N or with no visible key)
-    const float *dvec;    // [BH][Npad] D = rowsum(dO o O) (0 for rows past N)
-    float *dqacc;         // [BH][N][D] fp32, zeroed by bwd_pre
-    void *dk;             // [BH][N][D] 16-bit
-    void *dv;             // [BH][N][D] 16-bit
-    const uint8_t *mask;  // [nkb][nkb] block mask (kSparse)
-    int N;
-    int Npad;             // N rounded up to 128: row pitch of lse2 and dvec
+    const float *lse2;    // [BH][Npad] LSE * log2(e) (+inf for rows past Nq or with no visible key)
+    const float *dvec;    // [BH][Npad] D = rowsum(dO o O) (0 for rows past Nq)
+    float *dqacc;         // [BH][Nq][D] fp32, zeroed by bwd_pre
+    void *dk;             // [BH][Nk][D] 16-bit
+    void *dv;             // [BH][Nk][D] 16-bit
+    const uint8_t *mask;  // [ceil(Nq/128)][nkb] block mask (kSparse)
+    const float *alibi;   // [H] ALiBi slopes (natural-log units of the score), ALIBI kernels only
+    int Nq, Nk;           // query rows and keys per (b, h)
+    int off, wl, wr;      // visibility band (see band_any)
+    int H;                // heads (head of batch-head bh: bh % H)
+    int Npad;             // Nq rounded up to 128: row pitch of lse2 and dvec
     int nkb;              // key blocks (and mask blocks) of 128
     int nqt;              // query tiles of BM rows
     int nbh;              // batch x heads
@@ -115,7 +118,9 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict_
 template <int BM>
 __device__ __forceinline__ bool qtile_kept(const BwdParams &p, int i, int j) {
     if (i >= p.nqt) return false;
-    if ((p.mode & kCausal) && (i + 1) * BM <= j * 128) return false;   // every query precedes every key
+    const int q0 = i * BM, k0 = j * 128;
+    const int q1 = min(q0 + BM - 1, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
+    if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
     if ((p.mode & kSparse) && p.mask[static_cast<size_t>((i * BM) / 128) * p.nkb + j] == 0) return false;
     return true;
 }
@@ -213,7 +218,7 @@ struct BwdCfg {
 
 constexpr int kErrSmemAlign = 5;   // matches FA_ERR_CUDA
 
-template <int D, int NS, bool BF16>
+template <int D, int NS, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(512, 1)
             const int qh = warp >> 2;           // query half
             const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
             const int r = qd * 32 + lane;       // key row within the block
+            const int key = j * 128 + r;
             const float c = p.scale_log2;
             QIter<BM> it;
             int i;
@@ -437,18 +443,31 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
                 const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
                 const float4 *dd4 = lse4 + BM / 4;
-                const bool diag = (p.mode & kCausal) && i == j;
                 // phase A: P^T = 2^(S^T * scale * log2 e - LSE * log2 e), masked,
                 // rounded to 16 bits (kept packed in registers for phase B) and
                 // written over the S^T columns already read
                 const int q0 = 64 * qh;
+                // queries q0 + kk of this thread's half that see key `key`: lo <= kk <= hi
+                // (key q + off - wl .. q + off + wr); keys past Nk see none
+                const int qk = key - p.off - (i * BM + q0);     // |values| < 2^30 (Nq, Nk <= 2^28)
+                int lo = max(qk - p.wr, -1);
+                const int hi = min(qk + p.wl, 64);
+                if (key >= p.Nk) lo = 64;
+                const bool masked = __any_sync(0xffffffffu, lo > 0 || hi < 63);
                 uint32_t pk[32];
                 {
                     uint32_t sr[64];
                     tmem_ld32(tmem + lane_off + C::kColS + q0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                     tmem_ld32(tmem + lane_off + C::kColS + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                     tmem_ld_wait();
-                    const int lim = diag ? r - q0 : -1;    // queries q0 + kk with kk < lim precede key r
+                    if constexpr (ALIBI) {
+                        // score + bias / scale, bias = -slope |q + off - key|
+                        const float sl = -p.alibi[bh % p.H] / p.scale;
+                        const float base = static_cast<float>(-qk);
+#pragma unroll
+                        for (int kk = 0; kk < 64; ++kk)
+                            sr[kk] = __float_as_uint(fmaf(sl, fabsf(base + static_cast<float>(kk)), __uint_as_float(sr[kk])));
+                    }
 #pragma unroll
                     for (int k4 = 0; k4 < 16; ++k4) {
                         const float4 l4 = lse4[q0 / 4 + k4];
@@ -456,12 +475,18 @@ __global__ void __launch_bounds__(512, 1)
                         float x1 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 1]), c, -l4.y));
                         float x2 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 2]), c, -l4.z));
                         float x3 = ex2(fmaf(__uint_as_float(sr[4 * k4 + 3]), c, -l4.w));
-                        if (4 * k4 < lim) x0 = 0.f;
-                        if (4 * k4 + 1 < lim) x1 = 0.f;
-                        if (4 * k4 + 2 < lim) x2 = 0.f;
-                        if (4 * k4 + 3 < lim) x3 = 0.f;
                         pk[2 * k4] = pack2<BF16>(x0, x1);
                         pk[2 * k4 + 1] = pack2<BF16>(x2, x3);
+                    }
+                }
+                if (masked) {
+                    // zero the 16-bit P of queries outside [lo, hi] (element 2k in the low half)
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        uint32_t keep = 0xffffffffu;
+                        if (2 * k < lo || 2 * k > hi) keep &= 0xffff0000u;
+                        if (2 * k + 1 < lo || 2 * k + 1 > hi) keep &= 0x0000ffffu;
+                        pk[k] &= keep;
                     }
                 }
                 tmem_st32(tmem + lane_off + C::kColS + q0, pk);
@@ -523,12 +548,12 @@ __global__ void __launch_bounds__(512, 1)
     #pragma unroll
                             for (int k = 0; k < 32; ++k) v[k] = 0u;
                         }
-                        if (key < p.N) {
+                        if (key < p.Nk) {
                             uint32_t pk[16];
     #pragma unroll
                             for (int k = 0; k < 16; ++k)
                                 pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-                            uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D + 32 * ch) * 2);
+                            uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.Nk + key) * D + 32 * ch) * 2);
     #pragma unroll
                             for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                         }
@@ -557,8 +582,8 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarDqFree));
                 if (row_lane) {
-                    float *acc = p.dqacc + (static_cast<size_t>(bh) * p.N + static_cast<size_t>(i) * BM) * D + dcol;
-                    const int lim = p.N - i * BM;
+                    float *acc = p.dqacc + (static_cast<size_t>(bh) * p.Nq + static_cast<size_t>(i) * BM) * D + dcol;
+                    const int lim = p.Nq - i * BM;
 #pragma unroll
                     for (int k = 0; k < BM; ++k)
                         if (k < lim) atomicAdd(acc + k * D, __uint_as_float(v[k]));

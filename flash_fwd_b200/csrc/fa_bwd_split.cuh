@@ -57,7 +57,7 @@ struct BwdSplitCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(320, 1)
     bwd_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -292,13 +292,27 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             const float4 *lse4 = reinterpret_cast<const float4 *>(smem + C::kStatOff + s * 2 * C::kStatBytes);
             const float4 *dd4 = lse4 + BM / 4;
-            const bool need_causal = (p.mode & kCausal) && (i * BM < j * 128 + 127);
+            // queries i * BM + kk that see key `key`: lo <= kk <= hi (key q + off - wl ..
+            // q + off + wr); keys past Nk see none
+            const int qk = key - p.off - i * BM;     // |values| < 2^30 (Nq, Nk <= 2^28)
+            int lo = max(qk - p.wr, -1);
+            const int hi = min(qk + p.wl, BM);
+            if (key >= p.Nk) lo = BM;
+            const bool masked = __any_sync(0xffffffffu, lo > 0 || hi < BM - 1);
 #pragma unroll 1
             for (int ch = 0; ch < BM / 32; ++ch) {
                 uint32_t sr[32], pr[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32 * ch, sr);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, pr);
                 tmem_ld_wait();
+                if constexpr (ALIBI) {
+                    // score + bias / scale, bias = -slope |q + off - key|
+                    const float sl = -p.alibi[bh % p.H] / p.scale;
+                    const float base = static_cast<float>(-qk + 32 * ch);
+#pragma unroll
+                    for (int kk = 0; kk < 32; ++kk)
+                        sr[kk] = __float_as_uint(fmaf(sl, fabsf(base + static_cast<float>(kk)), __uint_as_float(sr[kk])));
+                }
                 if (ch == BM / 32 - 1) {
                     tc_fence_before();
                     mbar_arrive(bar(C::kBarSdpEmpty));
@@ -315,7 +329,7 @@ __global__ void __launch_bounds__(320, 1)
                     for (int e = 0; e < 4; ++e) {
                         const int kk = 4 * k4 + e;
                         float pv = ex2(fmaf(__uint_as_float(sr[kk]), c, -lv[e]));
-                        if (need_causal && key > i * BM + 32 * ch + kk) pv = 0.f;
+                        if (masked && (32 * ch + kk < lo || 32 * ch + kk > hi)) pv = 0.f;
                         pp[e] = pv;
                         ds[e] = pv * (__uint_as_float(pr[kk]) - dv[e]);
                     }
@@ -366,17 +380,17 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(bar(C::kBarDqEmpty));
-            float *accb = p.dqacc + static_cast<size_t>(bh) * p.N * D;
+            float *accb = p.dqacc + static_cast<size_t>(bh) * p.Nq * D;
             if constexpr (DQT) {
                 const int dcol = h * DH + t;
 #pragma unroll
                 for (int k = 0; k < BM; ++k) {
                     const int q = i * BM + k;
-                    if (q < p.N) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
+                    if (q < p.Nq) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
                 }
             } else {
                 const int q = i * BM + t;
-                if (q < p.N) {
+                if (q < p.Nq) {
                     float4 *dst = reinterpret_cast<float4 *>(accb + static_cast<size_t>(q) * D + h * DH);
 #pragma unroll
                     for (int k = 0; k < DH / 4; ++k)
@@ -411,12 +425,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] = 0u;
                 }
-                if (key < p.N) {
+                if (key < p.Nk) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
                         pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.N + key) * D +
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.Nk + key) * D +
                                                                   h * DH + 32 * ch) * 2);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);

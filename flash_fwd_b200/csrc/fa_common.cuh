@@ -43,6 +43,21 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
 // ---------------------------------------------------------------------------
+// Visibility band.  Query row r (of Nq) sees keys r + off - wl .. r + off + wr
+// (of Nk), off = Nk - Nq (the last query meets the last key); causal is
+// wr = 0, an unbounded side is kUnbounded.  A block-sparse mask, when given,
+// further removes whole 128 x 128 blocks.
+// ---------------------------------------------------------------------------
+// Nq, Nk <= kMaxRows keep every band expression within int.
+constexpr int kUnbounded = 1 << 29;
+constexpr int kMaxRows = 1 << 28;
+
+// Does any query row in [q0, q1] see any key in [k0, k1]?
+__device__ __forceinline__ bool band_any(int q0, int q1, int k0, int k1, int off, int wl, int wr) {
+    return k0 <= q1 + off + wr && k1 >= q0 + off - wl;
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -46,21 +46,27 @@ namespace fa {
 enum MaskMode : int { kDense = 0, kCausal = 1, kSparse = 2 };
 
 struct FwdParams {
-    void *o;                  // [BH][N][D] 16-bit
-    float *lse;               // [BH][N]
+    void *o;                  // [BH][Nq][D] 16-bit
+    float *lse;               // [BH][Nq]
     const uint8_t *mask;      // [nqb][nkb] block mask (kSparse)
-    int N;
+    const float *alibi;       // [H] ALiBi slopes (natural-log units of the score), ALIBI kernels only
+    int Nq, Nk;               // query rows and keys per (b, h)
+    int off, wl, wr;          // visibility band (see band_any)
     int nqb;                  // query blocks of 128 rows
     int nkb;                  // key blocks of 128 keys
     int nbh;                  // batch x heads
-    int mode;                 // kCausal | kSparse bits
+    int H;                    // heads (head of batch-head bh: bh % H)
+    int mode;                 // kCausal (heaviest-first order) | kSparse bits
+    float scale;
     float scale_log2;         // scale * log2(e)
 };
 
 // Is key block j visible at all from query block rb?
 __device__ __forceinline__ bool block_kept(const FwdParams &p, int rb, int j) {
     if (rb >= p.nqb || j >= p.nkb) return false;
-    if ((p.mode & kCausal) && j > rb) return false;
+    const int q0 = rb * 128, k0 = j * 128;
+    const int q1 = min(q0 + 127, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
+    if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
     if ((p.mode & kSparse) && p.mask[static_cast<size_t>(rb) * p.nkb + j] == 0) return false;
     return true;
 }
@@ -145,7 +151,7 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int D, int NQ, int NSK, int NSV, bool BF16>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -389,14 +395,21 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
             tmem_ld_wait();
             float *sv = reinterpret_cast<float *>(r);
-            const bool diag = (p.mode & kCausal) && j == rb;
-            const bool tail = (j == p.nkb - 1) && (p.N & 127);
-            if (diag || tail) {
-                int lim = tail ? (p.N - j * 128) : 128;
-                if (diag) lim = min(lim, row_local + 1);
+            // this row's visible keys within the tile: [lo, hi]
+            const int rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
+            const int lo = max(rk - p.wl, -1);
+            const int hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
+            if constexpr (ALIBI) {
+                // score + bias / scale, bias = -slope |row + off - key|
+                const float sl = -p.alibi[bh % p.H] / p.scale;
+                const float base = static_cast<float>(rk);
+#pragma unroll
+                for (int k = 0; k < 128; ++k) sv[k] = fmaf(sl, fabsf(base - static_cast<float>(k)), sv[k]);
+            }
+            if (__any_sync(0xffffffffu, lo > 0 || hi < 127)) {
 #pragma unroll
                 for (int k = 0; k < 128; ++k)
-                    if (k >= lim) sv[k] = -INFINITY;
+                    if (k < lo || k > hi) sv[k] = -INFINITY;
             }
             // row max: four independent chains of three-input max
             float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
@@ -477,11 +490,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         if (ok && cnt > 0) ok = wait_bar(bar(C::kBarOFull + t), 0, abort_flag);
         tc_fence_after();
         if (rb < p.nqb && ok) {
-            const bool valid = row < p.N;
+            const bool valid = row < p.Nq;
             const float l_o = BF16 ? l_r : l;
             const float inv_l = (cnt > 0 && l_o > 0.f) ? 1.0f / l_o : 0.0f;
             uint8_t *orow = reinterpret_cast<uint8_t *>(p.o) +
-                            (static_cast<size_t>(bh) * p.N + (valid ? row : 0)) * D * 2;
+                            (static_cast<size_t>(bh) * p.Nq + (valid ? row : 0)) * D * 2;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -507,7 +520,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             if (valid) {
                 const float lse = (cnt > 0 && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f
                                                         : -INFINITY;
-                p.lse[static_cast<size_t>(bh) * p.N + row] = lse;
+                p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
             }
         }
     }

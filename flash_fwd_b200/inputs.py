@@ -74,3 +74,23 @@ def sample_key_blocks(nb, count, seed, head):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+def make_qkv_cross(B, H, Nq, Nk, d, dtype="bf16", seed=0, qk_std=1.0):
+    """Q, dO [B, H, Nq, d] and K, V [B, H, Nk, d] CPU tensors of ``dtype``; the
+    same recipe as make_qkv (draw order Q, K, V, dO)."""
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    do = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    if qk_std != 1.0:
+        q, k = q * qk_std, k * qk_std
+    t = DTYPES[dtype]
+    return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous(), do.to(t).contiguous()
+
+
+def alibi_slopes(H):
+    """The geometric head slopes 2^(-8 (h + 1) / H) commonly used with ALiBi (fp32 [H])."""
+    return torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32)
+

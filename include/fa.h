@@ -21,7 +21,8 @@
  *            五; a multiple of 16 per "原理概览" section 3.4).
  * N          any N >= 1; a ragged last tile is masked.  N is both the query
  *            and the key length.
- * scale      the softmax scale, supplied by the caller (usually 1/sqrt(d)).
+ * scale      the softmax scale, supplied by the caller (usually 1/sqrt(d));
+ *            it must be positive and finite, else FA_ERR_INVALID_ARG.
  * causal     nonzero: query i sees key j only when j <= i ("深度解析" 五).
  * stream     a cudaStream_t passed as void*; NULL means the legacy default
  *            stream.  Every call is asynchronous on it.
@@ -57,7 +58,7 @@ typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
 
 typedef enum {
     FA_OK = 0,
-    FA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad flag, non-finite scale */
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad flag, scale not positive and finite */
     FA_ERR_UNSUPPORTED = 2,  /* d not in {64, 128, 256}, or a size beyond the kernel limits */
     FA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
     FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than fa_bwd_workspace_bytes() */
@@ -93,6 +94,30 @@ FA_API int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void 
                               void *stream);
 
 /*
+ * General forward: query and key lengths may differ, and the built-in mask
+ * modes other than causal ("深度解析" section 五: causal, sliding window,
+ * ALiBi) are available.
+ *   q, o      [B][H][Nq][d];  k, v [B][H][Nk][d];  lse [B][H][Nq]
+ *   alignment bottom-right: query i meets key i + (Nk - Nq) on the diagonal
+ *             (the same as top-left when Nq == Nk)
+ *   causal    key j visible to query i only if j <= i + Nk - Nq
+ *   window    key j visible only if i + Nk - Nq - window_left <= j <=
+ *             i + Nk - Nq + window_right; a negative side is unbounded
+ *             (window_left = window_right = -1: no window); combined with
+ *             causal the right side is 0
+ *   alibi_slopes  DEVICE float [H] (4-byte aligned) or NULL: adds
+ *             -alibi_slopes[h] * |i + Nk - Nq - j| to the scaled score
+ *             scale * q_i . k_j of head h (every batch shares the slopes)
+ *   block_mask    DEVICE uint8 [ceil(Nq/FA_BLOCK)][ceil(Nk/FA_BLOCK)] or NULL
+ * A query row that sees no key gets O = 0 and LSE = -inf (rows 0 .. Nq-Nk-1
+ * under causal when Nq > Nk, for instance).  Nq, Nk <= 2^28.
+ */
+FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                     int window_left, int window_right, const float *alibi_slopes,
+                     const uint8_t *block_mask, int dtype, void *stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: two fp32 per-row statistics
  * (LSE * log2 e and D = rowsum(dO * O)), each [B][H][Npad] with N padded up
  * to a multiple of FA_BLOCK, then an fp32 dQ accumulator [B][H][N][d].
@@ -114,6 +139,21 @@ FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, co
                   void *workspace, size_t workspace_bytes,
                   int B, int H, int N, int d, float scale, int causal, int dtype,
                   void *stream);
+
+/* Workspace of fa_bwd_ex: it depends on the query side only (Nq rows). */
+FA_API size_t fa_bwd_ex_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+
+/*
+ * General backward, the arguments and layouts of fa_fwd_ex: dq [B][H][Nq][d],
+ * dk, dv [B][H][Nk][d].  Reads the lse fa_fwd_ex wrote with the same
+ * arguments.  Keys that no query sees get zero dk, dv.
+ */
+FA_API int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                     const float *lse, void *dq, void *dk, void *dv,
+                     void *workspace, size_t workspace_bytes,
+                     int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                     int window_left, int window_right, const float *alibi_slopes,
+                     const uint8_t *block_mask, int dtype, void *stream);
 
 /* Block-sparse backward; block_mask as for fa_fwd_blocksparse. */
 FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,

@@ -54,6 +54,8 @@ def _fwd(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, N=128, d=64, scale=0.125, causal=0
     (dict(dtype=7), INVALID),
     (dict(scale=float("nan")), INVALID),
     (dict(scale=float("inf")), INVALID),
+    (dict(scale=0.0), INVALID),
+    (dict(scale=-0.125), INVALID),
     (dict(q=NULL), INVALID),
     (dict(lse=NULL), INVALID),
     (dict(k=M), MISALIGNED),
