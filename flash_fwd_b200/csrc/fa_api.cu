@@ -102,6 +102,8 @@ struct Problem {
         return win_right < 0 ? fa::kUnbounded : (win_right < fa::kUnbounded ? win_right : fa::kUnbounded);
     }
     int mode() const { return (causal ? fa::kCausal : 0) | (mask ? fa::kSparse : 0); }
+    // square, windowless, unbiased problems run the plain (non-GENERAL) kernels
+    bool general() const { return Nq != Nk || win_left >= 0 || win_right >= 0 || alibi != nullptr; }
 };
 
 Problem square(int B, int H, int N, int d, float scale, int causal, const uint8_t *mask, int dtype) {
@@ -119,11 +121,11 @@ int check_problem(const Problem &pr) {
     return FA_OK;
 }
 
-template <int D, int NQ, int NSK, int NSV, bool BF16, bool ALIBI>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
 int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const fa::FwdParams &p,
                int BH, cudaStream_t stream) {
     using C = fa::FwdCfg<D, NQ, NSK, NSV>;
-    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, ALIBI>;
+    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, GENERAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     const long long ctas = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
@@ -134,13 +136,13 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <bool BF16, bool ALIBI>
+template <bool BF16, bool GENERAL>
 int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                  const fa::FwdParams &p, int BH, cudaStream_t s) {
     switch (d) {
-        case 64: return launch_fwd<64, 2, 6, 4, BF16, ALIBI>(mq, mk, mv, p, BH, s);
-        case 128: return launch_fwd<128, 2, 3, 2, BF16, ALIBI>(mq, mk, mv, p, BH, s);
-        case 256: return launch_fwd<256, 1, 1, 1, BF16, ALIBI>(mq, mk, mv, p, BH, s);
+        case 64: return launch_fwd<64, 2, 6, 4, BF16, GENERAL>(mq, mk, mv, p, BH, s);
+        case 128: return launch_fwd<128, 2, 3, 2, BF16, GENERAL>(mq, mk, mv, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, 1, BF16, GENERAL>(mq, mk, mv, p, BH, s);
         default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -175,11 +177,12 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     p.scale = pr.scale;
     p.scale_log2 = pr.scale * kLog2e;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool general = pr.general();
     if (pr.dtype == FA_BF16)
-        return pr.alibi ? dispatch_fwd<true, true>(pr.d, mq, mk, mv, p, BH, s)
-                        : dispatch_fwd<true, false>(pr.d, mq, mk, mv, p, BH, s);
-    return pr.alibi ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, p, BH, s)
-                    : dispatch_fwd<false, false>(pr.d, mq, mk, mv, p, BH, s);
+        return general ? dispatch_fwd<true, true>(pr.d, mq, mk, mv, p, BH, s)
+                       : dispatch_fwd<true, false>(pr.d, mq, mk, mv, p, BH, s);
+    return general ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, p, BH, s)
+                   : dispatch_fwd<false, false>(pr.d, mq, mk, mv, p, BH, s);
 }
 
 
@@ -264,22 +267,22 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuf
     return launch_bwd_post<BF16>(dqacc, bb.dq, static_cast<long long>(BH) * pr.Nq * D, pr.scale, stream);
 }
 
-template <bool BF16, bool ALIBI>
+template <bool BF16, bool GENERAL>
 int dispatch_bwd(const BwdBuffers &bb, const Problem &pr, cudaStream_t s) {
     switch (pr.d) {
         case 64: {
             using C = fa::BwdCfg<64, 3>;
-            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16, ALIBI>, C::kSmemBytes, C::kThreads, 1, bb,
+            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16, GENERAL>, C::kSmemBytes, C::kThreads, 1, bb,
                                              pr, s);
         }
         case 128: {
             using C = fa::BwdCfg<128, 2>;
-            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16, ALIBI>, C::kSmemBytes, C::kThreads, 1,
+            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16, GENERAL>, C::kSmemBytes, C::kThreads, 1,
                                               bb, pr, s);
         }
         case 256: {
             using C = fa::BwdSplitCfg<256, 64, 2, 1, 2, true>;
-            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, ALIBI>,
+            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, GENERAL>,
                                              C::kSmemBytes, C::kThreads, 2, bb, pr, s);
         }
         default: return FA_ERR_UNSUPPORTED;
@@ -299,9 +302,10 @@ int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, vo
     if (!bb.workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(bb.workspace)) return FA_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool general = pr.general();
     if (pr.dtype == FA_BF16)
-        return pr.alibi ? dispatch_bwd<true, true>(bb, pr, s) : dispatch_bwd<true, false>(bb, pr, s);
-    return pr.alibi ? dispatch_bwd<false, true>(bb, pr, s) : dispatch_bwd<false, false>(bb, pr, s);
+        return general ? dispatch_bwd<true, true>(bb, pr, s) : dispatch_bwd<true, false>(bb, pr, s);
+    return general ? dispatch_bwd<false, true>(bb, pr, s) : dispatch_bwd<false, false>(bb, pr, s);
 }
 
 // ---------------------------------------------------------------- fa_bwd_noalloc

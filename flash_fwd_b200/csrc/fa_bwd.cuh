@@ -42,7 +42,7 @@ struct BwdParams {
     void *dk;             // [BH][Nk][D] 16-bit
     void *dv;             // [BH][Nk][D] 16-bit
     const uint8_t *mask;  // [ceil(Nq/128)][nkb] block mask (kSparse)
-    const float *alibi;   // [H] ALiBi slopes (natural-log units of the score), ALIBI kernels only
+    const float *alibi;   // [H] ALiBi slopes (natural-log units of the score) or null (GENERAL kernels)
     int Nq, Nk;           // query rows and keys per (b, h)
     int off, wl, wr;      // visibility band (see band_any)
     int H;                // heads (head of batch-head bh: bh % H)
@@ -115,18 +115,25 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict_
 // ---------------------------------------------------------------------------
 // bwd_main
 // ---------------------------------------------------------------------------
-template <int BM>
+// GENERAL kernels handle Nq != Nk, windows and ALiBi through the visibility
+// band; the others serve square problems (dense, causal, block-sparse) with
+// the plain causal test, which keeps their inner loops as lean as possible.
+template <int BM, bool GENERAL>
 __device__ __forceinline__ bool qtile_kept(const BwdParams &p, int i, int j) {
     if (i >= p.nqt) return false;
-    const int q0 = i * BM, k0 = j * 128;
-    const int q1 = min(q0 + BM - 1, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
-    if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
+    if constexpr (GENERAL) {
+        const int q0 = i * BM, k0 = j * 128;
+        const int q1 = min(q0 + BM - 1, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
+        if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
+    } else {
+        if ((p.mode & kCausal) && (i + 1) * BM <= j * 128) return false;   // every query precedes every key
+    }
     if ((p.mode & kSparse) && p.mask[static_cast<size_t>((i * BM) / 128) * p.nkb + j] == 0) return false;
     return true;
 }
 
 // Walks the query tiles that see key block j, in increasing order (warp-collective).
-template <int BM>
+template <int BM, bool GENERAL>
 struct QIter {
     int base = -32;
     uint32_t b = 0;
@@ -134,7 +141,7 @@ struct QIter {
         while (b == 0u) {
             base += 32;
             if (base >= p.nqt) return false;
-            b = __ballot_sync(0xffffffffu, qtile_kept<BM>(p, base + static_cast<int>(lane_id()), j));
+            b = __ballot_sync(0xffffffffu, qtile_kept<BM, GENERAL>(p, base + static_cast<int>(lane_id()), j));
         }
         const int k = __ffs(b) - 1;
         b &= b - 1;
@@ -218,7 +225,7 @@ struct BwdCfg {
 
 constexpr int kErrSmemAlign = 5;   // matches FA_ERR_CUDA
 
-template <int D, int NS, bool BF16, bool ALIBI>
+template <int D, int NS, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -288,7 +295,7 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
             __syncwarp();
-            QIter<BM> it;
+            QIter<BM, GENERAL> it;
             int i;
             while (it.next(p, j, i)) {
                 const int s = cnt % NS;
@@ -359,7 +366,7 @@ __global__ void __launch_bounds__(512, 1)
                     mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u, leader);
             };
 
-            QIter<BM> it;
+            QIter<BM, GENERAL> it;
             int i, in;
             bool have = it.next(p, j, i);
             if (have) {
@@ -432,7 +439,7 @@ __global__ void __launch_bounds__(512, 1)
             const int r = qd * 32 + lane;       // key row within the block
             const int key = j * 128 + r;
             const float c = p.scale_log2;
-            QIter<BM> it;
+            QIter<BM, GENERAL> it;
             int i;
             while (it.next(p, j, i)) {
                 const int s = cnt % NS;
@@ -449,18 +456,28 @@ __global__ void __launch_bounds__(512, 1)
                 const int q0 = 64 * qh;
                 // queries q0 + kk of this thread's half that see key `key`: lo <= kk <= hi
                 // (key q + off - wl .. q + off + wr); keys past Nk see none
-                const int qk = key - p.off - (i * BM + q0);     // |values| < 2^30 (Nq, Nk <= 2^28)
-                int lo = max(qk - p.wr, -1);
-                const int hi = min(qk + p.wl, 64);
-                if (key >= p.Nk) lo = 64;
-                const bool masked = __any_sync(0xffffffffu, lo > 0 || hi < 63);
+                int qk, lo, hi;
+                bool masked;
+                if constexpr (GENERAL) {
+                    qk = key - p.off - (i * BM + q0);     // |values| < 2^30 (Nq, Nk <= 2^28)
+                    lo = max(qk - p.wr, -1);
+                    hi = min(qk + p.wl, 64);
+                    if (key >= p.Nk) lo = 64;
+                    masked = __any_sync(0xffffffffu, lo > 0 || hi < 63);
+                } else {
+                    // square: the diagonal tile hides queries before the key
+                    qk = 0;
+                    hi = 64;
+                    lo = r - q0;
+                    masked = (p.mode & kCausal) && i == j;
+                }
                 uint32_t pk[32];
                 {
                     uint32_t sr[64];
                     tmem_ld32(tmem + lane_off + C::kColS + q0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                     tmem_ld32(tmem + lane_off + C::kColS + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                     tmem_ld_wait();
-                    if constexpr (ALIBI) {
+                    if (GENERAL && p.alibi) {
                         // score + bias / scale, bias = -slope |q + off - key|
                         const float sl = -p.alibi[bh % p.H] / p.scale;
                         const float base = static_cast<float>(-qk);
@@ -568,7 +585,7 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
             const bool row_lane = (D == 128) || (lane < 16);
             const int dcol = (D == 128) ? wq * 32 + lane : wq * 16 + (lane & 15);
-            QIter<BM> it;
+            QIter<BM, GENERAL> it;
             int i;
             while (it.next(p, j, i)) {
                 ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);

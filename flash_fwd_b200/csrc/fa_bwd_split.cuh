@@ -57,7 +57,7 @@ struct BwdSplitCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16, bool ALIBI>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(320, 1)
     bwd_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
         __syncwarp();
-        QIter<BM> it;
+        QIter<BM, GENERAL> it;
         int i;
         while (it.next(p, j, i)) {
             const int s = cnt % NS;
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(320, 1)
             }
         };
 
-        QIter<BM> it;
+        QIter<BM, GENERAL> it;
         int i, in;
         bool have = it.next(p, j, i);
         if (have) {
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(320, 1)
         const int r = warp * 32 + lane;     // key row within the block
         const int key = j * 128 + r;
         const float c = p.scale_log2;
-        QIter<BM> it;
+        QIter<BM, GENERAL> it;
         int i;
         while (it.next(p, j, i)) {
             const int s = cnt % NS;
@@ -294,18 +294,28 @@ __global__ void __launch_bounds__(320, 1)
             const float4 *dd4 = lse4 + BM / 4;
             // queries i * BM + kk that see key `key`: lo <= kk <= hi (key q + off - wl ..
             // q + off + wr); keys past Nk see none
-            const int qk = key - p.off - i * BM;     // |values| < 2^30 (Nq, Nk <= 2^28)
-            int lo = max(qk - p.wr, -1);
-            const int hi = min(qk + p.wl, BM);
-            if (key >= p.Nk) lo = BM;
-            const bool masked = __any_sync(0xffffffffu, lo > 0 || hi < BM - 1);
+            int qk, lo, hi;
+            bool masked;
+            if constexpr (GENERAL) {
+                qk = key - p.off - i * BM;     // |values| < 2^30 (Nq, Nk <= 2^28)
+                lo = max(qk - p.wr, -1);
+                hi = min(qk + p.wl, BM);
+                if (key >= p.Nk) lo = BM;
+                masked = __any_sync(0xffffffffu, lo > 0 || hi < BM - 1);
+            } else {
+                // square: queries before the key are hidden on the diagonal tiles
+                qk = 0;
+                hi = BM;
+                lo = key - i * BM;
+                masked = (p.mode & kCausal) && (i * BM < j * 128 + 127);
+            }
 #pragma unroll 1
             for (int ch = 0; ch < BM / 32; ++ch) {
                 uint32_t sr[32], pr[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32 * ch, sr);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, pr);
                 tmem_ld_wait();
-                if constexpr (ALIBI) {
+                if (GENERAL && p.alibi) {
                     // score + bias / scale, bias = -slope |q + off - key|
                     const float sl = -p.alibi[bh % p.H] / p.scale;
                     const float base = static_cast<float>(-qk + 32 * ch);
@@ -367,7 +377,7 @@ __global__ void __launch_bounds__(320, 1)
         // ------------------------------------------------------------ dQ drain
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int t = (warp & 3) * 32 + lane;   // TMEM lane: a d index (transposed form) or a query row
-        QIter<BM> it;
+        QIter<BM, GENERAL> it;
         int i;
         while (it.next(p, j, i)) {
             ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);

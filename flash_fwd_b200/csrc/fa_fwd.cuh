@@ -49,7 +49,7 @@ struct FwdParams {
     void *o;                  // [BH][Nq][D] 16-bit
     float *lse;               // [BH][Nq]
     const uint8_t *mask;      // [nqb][nkb] block mask (kSparse)
-    const float *alibi;       // [H] ALiBi slopes (natural-log units of the score), ALIBI kernels only
+    const float *alibi;       // [H] ALiBi slopes (natural-log units of the score) or null (GENERAL kernels)
     int Nq, Nk;               // query rows and keys per (b, h)
     int off, wl, wr;          // visibility band (see band_any)
     int nqb;                  // query blocks of 128 rows
@@ -61,19 +61,26 @@ struct FwdParams {
     float scale_log2;         // scale * log2(e)
 };
 
-// Is key block j visible at all from query block rb?
+// Is key block j visible at all from query block rb?  GENERAL kernels handle
+// Nq != Nk, windows and ALiBi through the visibility band; the others serve
+// square problems (dense, causal, block-sparse) with the plain causal test.
+template <bool GENERAL>
 __device__ __forceinline__ bool block_kept(const FwdParams &p, int rb, int j) {
     if (rb >= p.nqb || j >= p.nkb) return false;
-    const int q0 = rb * 128, k0 = j * 128;
-    const int q1 = min(q0 + 127, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
-    if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
+    if constexpr (GENERAL) {
+        const int q0 = rb * 128, k0 = j * 128;
+        const int q1 = min(q0 + 127, p.Nq - 1), k1 = min(k0 + 127, p.Nk - 1);
+        if (!band_any(q0, q1, k0, k1, p.off, p.wl, p.wr)) return false;
+    } else {
+        if ((p.mode & kCausal) && j > rb) return false;
+    }
     if ((p.mode & kSparse) && p.mask[static_cast<size_t>(rb) * p.nkb + j] == 0) return false;
     return true;
 }
 
 // Walks, in increasing order, the key blocks kept by at least one of the CTA's
 // NQ query blocks (rb0, rb0 + 1).  Warp-collective: all 32 lanes call next().
-template <int NQ>
+template <int NQ, bool GENERAL>
 struct KvIter {
     int base = -32;
     uint32_t b0 = 0, b1 = 0;
@@ -82,8 +89,8 @@ struct KvIter {
             base += 32;
             if (base >= p.nkb) return false;
             const int jj = base + static_cast<int>(lane_id());
-            b0 = __ballot_sync(0xffffffffu, block_kept(p, rb0, jj));
-            b1 = (NQ > 1) ? __ballot_sync(0xffffffffu, block_kept(p, rb0 + 1, jj)) : 0u;
+            b0 = __ballot_sync(0xffffffffu, block_kept<GENERAL>(p, rb0, jj));
+            b1 = (NQ > 1) ? __ballot_sync(0xffffffffu, block_kept<GENERAL>(p, rb0 + 1, jj)) : 0u;
         }
         const uint32_t u = b0 | b1;
         const int b = __ffs(u) - 1;
@@ -151,7 +158,7 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int D, int NQ, int NSK, int NSV, bool BF16, bool ALIBI>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 }
             }
             __syncwarp();
-            KvIter<NQ> it;
+            KvIter<NQ, GENERAL> it;
             int j;
             uint32_t f;
             int nk = 0, nv = 0;   // loads issued
@@ -290,7 +297,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                            (acc || k > 0) ? 1u : 0u, leader);
             };
 
-            KvIter<NQ> it;
+            KvIter<NQ, GENERAL> it;
             int j, jn;
             uint32_t f, fn;
             int cnt[NQ];
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         const float c = p.scale_log2;
         float m = -INFINITY, l = 0.f, l_r = 0.f;
         int cnt = 0;
-        KvIter<NQ> it;
+        KvIter<NQ, GENERAL> it;
         int j;
         uint32_t f;
         bool ok = true;
@@ -396,10 +403,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             tmem_ld_wait();
             float *sv = reinterpret_cast<float *>(r);
             // this row's visible keys within the tile: [lo, hi]
-            const int rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
-            const int lo = max(rk - p.wl, -1);
-            const int hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
-            if constexpr (ALIBI) {
+            int lo, hi, rk = 0;
+            if constexpr (GENERAL) {
+                rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
+                lo = max(rk - p.wl, -1);
+                hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
+            } else {
+                lo = -1;
+                hi = 127;
+                if ((p.mode & kCausal) && j == rb) hi = row_local;                    // diagonal tile
+                if (j == p.nkb - 1 && (p.Nk & 127)) hi = min(hi, (p.Nk & 127) - 1);  // key tail
+            }
+            if (GENERAL && p.alibi) {
                 // score + bias / scale, bias = -slope |row + off - key|
                 const float sl = -p.alibi[bh % p.H] / p.scale;
                 const float base = static_cast<float>(rk);
