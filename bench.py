@@ -50,7 +50,17 @@ WORKLOADS = {
     "sparse64k": dict(B=1, H=4, N=65536, d=64, dtype="bf16", causal=False, sparse=True, bwd=True,
                       density=0.2),
     "tiny": dict(B=1, H=2, N=128, d=64, dtype="f16", causal=False, sparse=False, bwd=True),
+    # the general entry points: a sliding window, a decoder chunk attending to
+    # a longer context, ALiBi (causal), all at the d = 128 sweep's size
+    "window128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True,
+                      window=(1024, 0)),
+    "cross128": dict(B=4, H=16, N=1024, Nk=8192, d=128, dtype="bf16", causal=True, sparse=False, bwd=True),
+    "alibi128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True, alibi=True),
 }
+
+
+def general(w):
+    return "Nk" in w or "window" in w or w.get("alibi", False)
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -81,6 +91,8 @@ def workload_flops(w, kept_blocks=None):
     from flash_fwd_b200 import accounting as acc
     if w["sparse"]:
         f = acc.sparse_fwd_flops(w["B"], w["H"], w["d"], kept_blocks)
+    elif "Nk" in w or "window" in w:
+        f = acc.general_fwd_flops(w["B"], w["H"], w["N"], w.get("Nk", w["N"]), w["d"], w["causal"], w.get("window"))
     else:
         f = acc.fwd_flops(w["B"], w["H"], w["N"], w["d"], w["causal"])
     b = 2.5 * f if w["bwd"] else 0.0
@@ -91,6 +103,9 @@ def describe(name, w):
     s = f"{name}: B={w['B']} H={w['H']} N={w['N']} d={w['d']} {w['dtype']}"
     s += " causal" if w["causal"] else ""
     s += f" block-sparse(128x128, diag + Bernoulli {w['density']})" if w["sparse"] else ""
+    s += f" Nk={w['Nk']}" if "Nk" in w else ""
+    s += f" window={w['window']}" if "window" in w else ""
+    s += " alibi" if w.get("alibi") else ""
     s += " fwd+bwd" if w["bwd"] else " fwd"
     return s
 
@@ -185,24 +200,35 @@ def make_inputs(w, seed, device):
     import torch
 
     from flash_fwd_b200 import inputs
-    q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=seed, with_dout=w["bwd"])
+    if "Nk" in w:
+        q, k, v, do = inputs.make_qkv_cross(w["B"], w["H"], w["N"], w["Nk"], w["d"], w["dtype"], seed=seed)
+    else:
+        q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=seed, with_dout=w["bwd"])
     mask = inputs.make_block_mask(w["N"], 128, w.get("density", 0.2), seed=seed) if w["sparse"] else None
-    host = dict(q=q, k=k, v=v, do=do, mask=mask)
+    slopes = inputs.alibi_slopes(w["H"]) if w.get("alibi") else None
+    host = dict(q=q, k=k, v=v, do=do, mask=mask, slopes=slopes)
     dev = {n: (t.to(device) if t is not None else None) for n, t in host.items()}
     dev["o"] = torch.empty_like(dev["q"])
     dev["lse"] = torch.empty((w["B"], w["H"], w["N"]), dtype=torch.float32, device=device)
     if w["bwd"]:
         import flash_fwd_b200 as fa
-        dev["dq"], dev["dk"], dev["dv"] = (torch.empty_like(dev["q"]) for _ in range(3))
-        dev["ws"] = torch.empty(fa.fa_bwd_workspace_bytes(w["B"], w["H"], w["N"], w["d"]), dtype=torch.uint8,
-                                device=device)
+        dev["dq"] = torch.empty_like(dev["q"])
+        dev["dk"], dev["dv"] = torch.empty_like(dev["k"]), torch.empty_like(dev["v"])
+        dev["ws"] = torch.empty(fa.fa_bwd_ex_workspace_bytes(w["B"], w["H"], w["N"], w.get("Nk", w["N"]), w["d"]),
+                                dtype=torch.uint8, device=device)
     return host, dev
 
 
 def step(w, t, stream):
     import flash_fwd_b200 as fa
     scale = 1.0 / w["d"] ** 0.5
-    if w["sparse"]:
+    if general(w):
+        fa.fa_fwd_ex(t["q"], t["k"], t["v"], t["o"], t["lse"], w["causal"], scale, w.get("window"), t["slopes"],
+                     t["mask"], stream)
+        if w["bwd"]:
+            fa.fa_bwd_ex(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"], t["ws"],
+                         w["causal"], scale, w.get("window"), t["slopes"], t["mask"], stream)
+    elif w["sparse"]:
         fa.fa_fwd_blocksparse(t["q"], t["k"], t["v"], t["o"], t["lse"], t["mask"], w["causal"], scale, stream)
         if w["bwd"]:
             fa.fa_bwd_blocksparse(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"],
@@ -223,19 +249,22 @@ def oracle_head_pass(host, w, head):
     import numpy as np
 
     import oracle
-    N, d = w["N"], w["d"]
+    N, Nk, d = w["N"], w.get("Nk", w["N"]), w["d"]
     b, h = divmod(head, w["H"])
-    sl = lambda t: t[b, h].reshape(1, N, d).double().numpy()  # noqa: E731
-    Q, K, V = sl(host["q"]), sl(host["k"]), sl(host["v"])
+    sl = lambda t, n: t[b, h].reshape(1, n, d).double().numpy()  # noqa: E731
+    Q, K, V = sl(host["q"], N), sl(host["k"], Nk), sl(host["v"], Nk)
     flags = (oracle.CAUSAL if w["causal"] else 0) | (oracle.SPARSE if w["sparse"] else 0)
     mask = host["mask"].numpy() if w["sparse"] else None
+    modes = dict(window=w.get("window"),
+                 slopes=None if host.get("slopes") is None else host["slopes"][h:h + 1].double().numpy())
     rows = np.arange(N, dtype=np.int32)
+    cols = np.arange(Nk, dtype=np.int32)
     t0 = time.perf_counter()
-    oracle.fwd_rows(Q, K, V, 1.0 / d ** 0.5, flags, mask, 128, rows)
+    oracle.fwd_rows(Q, K, V, 1.0 / d ** 0.5, flags, mask, 128, rows, **modes)
     if w["bwd"]:
-        DO = sl(host["do"])
-        oracle.bwd_dq_rows(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128)
-        oracle.bwd_dkdv_cols(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128)
+        DO = sl(host["do"], N)
+        oracle.bwd_dq_rows(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128, **modes)
+        oracle.bwd_dkdv_cols(Q, K, V, DO, 1.0 / d ** 0.5, cols, flags, mask, 128, **modes)
     return time.perf_counter() - t0
 
 
@@ -281,9 +310,13 @@ def run_reference(args, w, name):
 
 def make_inputs_cpu(w):
     from flash_fwd_b200 import inputs
-    q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=0, with_dout=w["bwd"])
+    if "Nk" in w:
+        q, k, v, do = inputs.make_qkv_cross(w["B"], w["H"], w["N"], w["Nk"], w["d"], w["dtype"], seed=0)
+    else:
+        q, k, v, do = inputs.make_qkv(w["B"], w["H"], w["N"], w["d"], w["dtype"], seed=0, with_dout=w["bwd"])
     mask = inputs.make_block_mask(w["N"], 128, w.get("density", 0.2), seed=0) if w["sparse"] else None
-    return dict(q=q, k=k, v=v, do=do, mask=mask), None
+    slopes = inputs.alibi_slopes(w["H"]) if w.get("alibi") else None
+    return dict(q=q, k=k, v=v, do=do, mask=mask, slopes=slopes), None
 
 
 # --------------------------------------------------------------------------

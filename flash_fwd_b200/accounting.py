@@ -6,6 +6,9 @@
   forward ("FlashAttention 深度解析", section 四).
 * Block-sparse: only kept 128 x 128 blocks count, 4*d*blk^2 per kept block per
   (batch, head) for the forward.
+* General problems (query and key lengths that differ, sliding windows):
+  4*d per visible (query, key) pair per (batch, head), the pairs counted
+  exactly from the visibility band (bottom-right aligned).
 * Minimum HBM bytes of the fused forward: read Q, K, V, write O (4*N*d*e) plus
   one fp32 LSE per row; of the backward: read Q, K, V, O, dO, LSE, D and write
   dQ, dK, dV (8*N*d*e + 8*N), before the fp32 dQ accumulator this design adds.
@@ -66,3 +69,23 @@ def sram_tile_bytes(Br, Bc, d, elem):
 def io_bound_elems(N, d, M):
     """The Theta(N^2 d^2 / M) HBM accesses of the tiled method (深度解析 section 三)."""
     return N * N * d * d / M
+
+
+def visible_pairs(Nq, Nk, causal=False, window=None):
+    """Number of (query, key) pairs a head attends to: query i sees keys
+    i + Nk - Nq - left .. i + Nk - Nq + right (right = 0 under causal; a
+    negative side is unbounded), clipped to 0 .. Nk - 1."""
+    import numpy as np
+    off = Nk - Nq
+    left, right = (-1, -1) if window is None else window
+    i = np.arange(Nq, dtype=np.int64)
+    lo = np.zeros(Nq, dtype=np.int64) if left < 0 else np.maximum(i + off - left, 0)
+    hi = np.full(Nq, Nk - 1, dtype=np.int64) if right < 0 else np.minimum(i + off + right, Nk - 1)
+    if causal:
+        hi = np.minimum(hi, i + off)
+    return int(np.maximum(hi - lo + 1, 0).sum())
+
+
+def general_fwd_flops(B, H, Nq, Nk, d, causal=False, window=None):
+    return 4.0 * B * H * d * visible_pairs(Nq, Nk, causal, window)
+

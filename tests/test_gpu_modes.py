@@ -122,3 +122,32 @@ def test_long_cross_attention_sampled():
         r_dk, r_dv = oracle.bwd_dkdv_cols(Q[sl], K[sl], V[sl], DO[sl], scale, cols, oracle.CAUSAL)
         for g, r in ((f(dq, nq)[h, rows], r_dq), (f(dk, nk)[h, cols], r_dk[0]), (f(dv, nk)[h, cols], r_dv[0])):
             assert np.abs(g - r).max() / max(np.abs(r).max(), GRAD_NORM_FLOOR) <= TOL_GRAD_REL
+
+
+@pytest.mark.parametrize("name", ["window128", "cross128", "alibi128"])
+def test_bench_workloads_sampled(name):
+    # the general workloads bench.py times, at their full size, on sampled rows and keys
+    w = dict(window128=dict(B=4, H=16, Nq=4096, Nk=4096, window=(1024, 0), alibi=False),
+             cross128=dict(B=4, H=16, Nq=1024, Nk=8192, window=None, alibi=False),
+             alibi128=dict(B=4, H=16, Nq=4096, Nk=4096, window=None, alibi=True))[name]
+    B, H, nq, nk, d = w["B"], w["H"], w["Nq"], w["Nk"], 128
+    q, k, v, do = inputs.make_qkv_cross(B, H, nq, nk, d, "bf16", seed=0)
+    scale = inputs.default_scale(d)
+    slopes = inputs.alibi_slopes(H) if w["alibi"] else None
+    o, lse, dq, dk, dv = _run(q, k, v, do, True, scale, window=w["window"], slopes=slopes)
+    f = lambda t, n: t.reshape(B * H, n, d).double().numpy()   # noqa: E731
+    Q, K, V, DO = f(q, nq), f(k, nk), f(v, nk), f(do, nq)
+    O, L = f(o, nq), lse.reshape(B * H, nq).double().numpy()
+    dQ, dK, dV = f(dq, nq), f(dk, nk), f(dv, nk)
+    for bh in (0, 37, 63):
+        rows = inputs.sample_rows(nq, 8, 0, bh).numpy()
+        cols = inputs.sample_rows(nk, 8, 7, bh).numpy()
+        sl = slice(bh, bh + 1)
+        kw = dict(window=w["window"], slopes=None if slopes is None else slopes[bh % H:bh % H + 1].double().numpy())
+        r_o, r_l = oracle.fwd_rows(Q[sl], K[sl], V[sl], scale, oracle.CAUSAL, rows=rows, **kw)
+        assert np.abs(O[bh, rows] - r_o[0]).max() <= TOL_O["bf16"]
+        assert np.abs(L[bh, rows] - r_l[0]).max() <= TOL_LSE
+        r_dq = oracle.bwd_dq_rows(Q[sl], K[sl], V[sl], DO[sl], scale, rows, oracle.CAUSAL, **kw)[0]
+        r_dk, r_dv = oracle.bwd_dkdv_cols(Q[sl], K[sl], V[sl], DO[sl], scale, cols, oracle.CAUSAL, **kw)
+        for g, r in ((dQ[bh, rows], r_dq), (dK[bh, cols], r_dk[0]), (dV[bh, cols], r_dv[0])):
+            assert np.abs(g - r).max() / max(np.abs(r).max(), GRAD_NORM_FLOOR) <= TOL_GRAD_REL
