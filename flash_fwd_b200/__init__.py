@@ -15,7 +15,8 @@ __all__ = [
     "FaError", "load_library", "library_path", "fa_fwd", "fa_fwd_blocksparse", "fa_bwd",
     "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status", "fa_last_timeout_site",
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
-    "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes",
+    "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes", "fa_bwd_deterministic",
+    "fa_bwd_deterministic_workspace_bytes",
 ]
 
 FA_BLOCK = 128
@@ -56,6 +57,9 @@ def load_library():
     lib.fa_bwd_ex_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_bwd_ex_workspace_bytes.restype = sz
     lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, i, vp, vp, i, vp]
+    lib.fa_bwd_deterministic_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_deterministic_workspace_bytes.restype = sz
+    lib.fa_bwd_deterministic.argtypes = list(lib.fa_bwd_ex.argtypes)
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -64,6 +68,7 @@ def load_library():
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
+               lib.fa_bwd_deterministic,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -91,7 +96,7 @@ def fa_version():
     return load_library().fa_version()
 
 
-PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post")
+PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post", "bwd_dq")
 
 
 def fa_profile_enable(on=True):
@@ -100,8 +105,8 @@ def fa_profile_enable(on=True):
 
 def fa_profile_read():
     """{kind: (milliseconds, launches)} summed since the last read."""
-    ms = (ctypes.c_float * 4)()
-    n = (ctypes.c_int * 4)()
+    ms = (ctypes.c_float * len(PROFILE_KINDS))()
+    n = (ctypes.c_int * len(PROFILE_KINDS))()
     _check(load_library().fa_profile_read(ms, n), "fa_profile_read")
     return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(PROFILE_KINDS)}
 
@@ -209,6 +214,23 @@ def fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=
     _check(rc, "fa_bwd_ex")
 
 
+def fa_bwd_deterministic_workspace_bytes(B, H, Nq, Nk, d):
+    return load_library().fa_bwd_deterministic_workspace_bytes(B, H, Nq, Nk, d)
+
+
+def fa_bwd_deterministic(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, window=None,
+                         alibi_slopes=None, block_mask=None, stream=None):
+    """fa_bwd_ex with bitwise reproducible outputs (dQ by a second sweep, no atomics)."""
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
+    wl, wr = _window(window)
+    rc = load_library().fa_bwd_deterministic(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)), wl, wr,
+        _ptr(alibi_slopes), _ptr(block_mask), _dtype(q), _stream(stream))
+    _check(rc, "fa_bwd_deterministic")
+
+
 def _general(q, k, window, alibi_slopes):
     return k.shape[2] != q.shape[2] or window is not None or alibi_slopes is not None
 
@@ -230,14 +252,19 @@ def attention_fwd(q, k, v, causal=False, scale=None, block_mask=None, stream=Non
 
 
 def attention_bwd(q, k, v, o, dout, lse, causal=False, scale=None, block_mask=None, workspace=None,
-                  stream=None, window=None, alibi_slopes=None):
-    """Allocates dQ, dK, dV (and the workspace unless given) and runs the backward."""
+                  stream=None, window=None, alibi_slopes=None, deterministic=False):
+    """Allocates dQ, dK, dV (and the workspace unless given) and runs the backward.
+    deterministic=True gives bitwise reproducible dQ (a second sweep instead of atomics)."""
     B, H, Nq, d = _shape(q)
     Nk = int(k.shape[2])
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
-        workspace = torch.empty(fa_bwd_ex_workspace_bytes(B, H, Nq, Nk, d), dtype=torch.uint8, device=q.device)
-    if _general(q, k, window, alibi_slopes):
+        nbytes = (fa_bwd_deterministic_workspace_bytes if deterministic else fa_bwd_ex_workspace_bytes)(B, H, Nq, Nk, d)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if deterministic:
+        fa_bwd_deterministic(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal, scale, window, alibi_slopes,
+                             block_mask, stream)
+    elif _general(q, k, window, alibi_slopes):
         fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal, scale, window, alibi_slopes, block_mask,
                   stream)
     elif block_mask is None:

@@ -11,6 +11,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_dq.cuh"
 #include "fa_bwd_split.cuh"
 #include "fa_fwd.cuh"
 
@@ -217,16 +218,38 @@ struct BwdBuffers {
     void *dq, *dk, *dv, *workspace;
 };
 
+// The deterministic dQ pass: one CTA per 128-row query tile (fa_bwd_dq.cuh).
+template <int D, bool BF16, bool GENERAL>
+int launch_bwd_dq(const BwdBuffers &bb, const Problem &pr, fa::BwdParams p, const CUtensorMap &mk,
+                  const CUtensorMap &mv, cudaStream_t stream) {
+    using C = fa::DqCfg<D>;
+    const int BH = static_cast<int>(pr.BH());
+    CUtensorMap mq, mdo;
+    int rc;
+    if ((rc = make_map(&mq, bb.q, D, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mdo, bb.dout, D, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
+    p.nqt = (pr.Nq + 127) / 128;
+    p.dq = bb.dq;
+    auto kern = fa::bwd_dq_kernel<D, BF16, GENERAL>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nqt));
+    ProfScope prof(4, stream);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 // Three launches: pre-pass, main kernel (Kernel: a bwd_kernel or bwd_split_kernel
-// instantiation, BM query rows per tile, `split` CTAs per key block), post-pass.
-template <int D, int BM, bool BF16, typename Kernel>
+// instantiation, BM query rows per tile, `split` CTAs per key block), then the
+// post-pass -- or, deterministic, the main kernel without dQ and the dQ pass.
+template <int D, int BM, bool BF16, bool GENERAL, typename Kernel>
 int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuffers &bb, const Problem &pr,
-               cudaStream_t stream) {
+               bool deterministic, cudaStream_t stream) {
     const int BH = static_cast<int>(pr.BH());
     const int Npad = fa::bwd_npad(pr.Nq);
     float *lse2 = static_cast<float *>(bb.workspace);
     float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
-    float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
+    float *dqacc = deterministic ? nullptr : dvec + static_cast<size_t>(BH) * Npad;
     int rc = launch_bwd_pre<D, BF16>(bb.o, bb.dout, bb.lse, lse2, dvec, dqacc, BH, pr.Nq, Npad, stream);
     if (rc != FA_OK) return rc;
     CUtensorMap mk, mv, mq, mdo;
@@ -238,6 +261,7 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuf
     p.lse2 = lse2;
     p.dvec = dvec;
     p.dqacc = dqacc;
+    p.dq = nullptr;
     p.dk = bb.dk;
     p.dv = bb.dv;
     p.mask = pr.mask;
@@ -264,32 +288,38 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuf
         kern<<<grid, threads, smem_bytes, stream>>>(mk, mv, mq, mdo, p);
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (deterministic) return launch_bwd_dq<D, BF16, GENERAL>(bb, pr, p, mk, mv, stream);
     return launch_bwd_post<BF16>(dqacc, bb.dq, static_cast<long long>(BH) * pr.Nq * D, pr.scale, stream);
 }
 
 template <bool BF16, bool GENERAL>
-int dispatch_bwd(const BwdBuffers &bb, const Problem &pr, cudaStream_t s) {
+int dispatch_bwd(const BwdBuffers &bb, const Problem &pr, bool det, cudaStream_t s) {
     switch (pr.d) {
         case 64: {
             using C = fa::BwdCfg<64, 3>;
-            return launch_bwd<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16, GENERAL>, C::kSmemBytes, C::kThreads, 1, bb,
-                                             pr, s);
+            return launch_bwd<64, 128, BF16, GENERAL>(fa::bwd_kernel<64, 3, BF16, GENERAL>, C::kSmemBytes,
+                                                      C::kThreads, 1, bb, pr, det, s);
         }
         case 128: {
             using C = fa::BwdCfg<128, 2>;
-            return launch_bwd<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16, GENERAL>, C::kSmemBytes, C::kThreads, 1,
-                                              bb, pr, s);
+            return launch_bwd<128, 128, BF16, GENERAL>(fa::bwd_kernel<128, 2, BF16, GENERAL>, C::kSmemBytes,
+                                                       C::kThreads, 1, bb, pr, det, s);
         }
         case 256: {
             using C = fa::BwdSplitCfg<256, 64, 2, 1, 2, true>;
-            return launch_bwd<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, GENERAL>,
-                                             C::kSmemBytes, C::kThreads, 2, bb, pr, s);
+            return launch_bwd<256, 64, BF16, GENERAL>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, GENERAL>,
+                                                      C::kSmemBytes, C::kThreads, 2, bb, pr, det, s);
         }
         default: return FA_ERR_UNSUPPORTED;
     }
 }
 
-int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, void *stream) {
+// Workspace of the deterministic backward: LSE * log2(e) and D only (no fp32
+// dQ accumulator).
+size_t bwd_det_workspace_bytes(long long BH, int Nq) { return 2 * static_cast<size_t>(BH) * fa::bwd_npad(Nq) * 4; }
+
+int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, void *stream,
+             bool deterministic = false) {
     if (!bb.q || !bb.k || !bb.v || !bb.o || !bb.dout || !bb.lse || !bb.dq || !bb.dk || !bb.dv)
         return FA_ERR_INVALID_ARG;
     int rc = check_problem(pr);
@@ -297,15 +327,18 @@ int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, vo
     const void *ptrs[] = {bb.q, bb.k, bb.v, bb.o, bb.dout, bb.lse, bb.dq, bb.dk, bb.dv};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
-    if (pr.BH() * (2LL * ((pr.Nk + 127) / 128)) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
-    const size_t need = fa::bwd_workspace_bytes(pr.BH(), pr.Nq, pr.d);
+    if (pr.BH() * (2LL * ((pr.Nk + 127) / 128)) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grids
+    if (pr.BH() * ((pr.Nq + 127LL) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    const size_t need = deterministic ? bwd_det_workspace_bytes(pr.BH(), pr.Nq)
+                                      : fa::bwd_workspace_bytes(pr.BH(), pr.Nq, pr.d);
     if (!bb.workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(bb.workspace)) return FA_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool general = pr.general();
+    const bool det = deterministic;
     if (pr.dtype == FA_BF16)
-        return general ? dispatch_bwd<true, true>(bb, pr, s) : dispatch_bwd<true, false>(bb, pr, s);
-    return general ? dispatch_bwd<false, true>(bb, pr, s) : dispatch_bwd<false, false>(bb, pr, s);
+        return general ? dispatch_bwd<true, true>(bb, pr, det, s) : dispatch_bwd<true, false>(bb, pr, det, s);
+    return general ? dispatch_bwd<false, true>(bb, pr, det, s) : dispatch_bwd<false, false>(bb, pr, det, s);
 }
 
 // ---------------------------------------------------------------- fa_bwd_noalloc
@@ -390,6 +423,21 @@ FA_API int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
     const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
     const Problem pr{B, H, Nq, Nk, d, scale, causal, window_left, window_right, alibi_slopes, block_mask, dtype};
     return bwd_impl(bb, workspace_bytes, pr, stream);
+}
+
+FA_API size_t fa_bwd_deterministic_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || (d != 64 && d != 128 && d != 256)) return 0;
+    return bwd_det_workspace_bytes(static_cast<long long>(B) * H, Nq);
+}
+
+FA_API int fa_bwd_deterministic(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                                const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                                size_t workspace_bytes, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                                int window_left, int window_right, const float *alibi_slopes,
+                                const uint8_t *block_mask, int dtype, void *stream) {
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    const Problem pr{B, H, Nq, Nk, d, scale, causal, window_left, window_right, alibi_slopes, block_mask, dtype};
+    return bwd_impl(bb, workspace_bytes, pr, stream, true);
 }
 
 FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const void *dout,

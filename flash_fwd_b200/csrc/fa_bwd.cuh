@@ -21,6 +21,9 @@
 //                                  (tcgen05, TMEM), then fp32 atomics into the
 //                                   accumulator by the drain warps.
 //   bwd_post  dQ = scale * accumulator, rounded to the 16-bit type.
+// The deterministic backward passes a null accumulator: bwd_main then computes
+// dK, dV only, and the dQ pass of fa_bwd_dq.cuh replaces the atomics and
+// bwd_post.
 //
 // Warp roles of bwd_main: warps 0-3 softmax-grad (and the dV epilogue), warps
 // 4-7 dQ drain (and the dK epilogue), warp 8 TMA producer (also stages the
@@ -38,7 +41,8 @@ namespace fa {
 struct BwdParams {
     const float *lse2;    // [BH][Npad] LSE * log2(e) (+inf for rows past Nq or with no visible key)
     const float *dvec;    // [BH][Npad] D = rowsum(dO o O) (0 for rows past Nq)
-    float *dqacc;         // [BH][Nq][D] fp32, zeroed by bwd_pre
+    float *dqacc;         // [BH][Nq][D] fp32, zeroed by bwd_pre; null: the key-block kernels skip dQ
+    void *dq;             // [BH][Nq][D] 16-bit (written by the deterministic dQ pass)
     void *dk;             // [BH][Nk][D] 16-bit
     void *dv;             // [BH][Nk][D] 16-bit
     const uint8_t *mask;  // [ceil(Nq/128)][nkb] block mask (kSparse)
@@ -82,9 +86,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint4 *__restrict__ 
             acc = fmaf(x.x, y.x, acc);
             acc = fmaf(x.y, y.y, acc);
         }
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        dqacc[(row * D + part * 8) / 4] = z;
-        dqacc[(row * D + part * 8) / 4 + 1] = z;
+        if (dqacc) {
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            dqacc[(row * D + part * 8) / 4] = z;
+            dqacc[(row * D + part * 8) / 4 + 1] = z;
+        }
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -356,14 +362,18 @@ __global__ void __launch_bounds__(512, 1)
                     mma_ts(tmem + C::kColDV, tmem + C::kColS + 8 * k + 32 * (k >> 2), ddO_mn.at(s * C::kQTile + k * 2048),
                            kIdKV, (acc || k > 0) ? 1u : 0u, leader);
             };
+            const bool with_dq = p.dqacc != nullptr;   // else the deterministic dQ pass computes dQ
             auto issue_dk_dq = [&](int s, bool acc) {
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)    // dK += dS^T Q_i
                     mma_ss(tmem + C::kColDK, ddS_k.at((k >> 2) * C::kChunk + (k & 3) * 32),
                            dQ_mn.at(s * C::kQTile + k * 2048), kIdKV, (acc || k > 0) ? 1u : 0u, leader);
+                if (with_dq) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)          // dQ^T (D x BM) = K_j^T dS^T, over the 128 keys
-                    mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u, leader);
+                    for (int k = 0; k < 8; ++k)      // dQ^T (D x BM) = K_j^T dS^T, over the 128 keys
+                        mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u,
+                               leader);
+                }
             };
 
             QIter<BM, GENERAL> it;
@@ -407,12 +417,13 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
                 {
                     issue_dk_dq(s, cnt > 0);
-                    mma_commit(bar(C::kBarDqFull), leader);
+                    if (with_dq) mma_commit(bar(C::kBarDqFull), leader);
                     mma_commit(bar(C::kBarQEmpty + s), leader);
                 }
                 __syncwarp();
                 if (have_n) {
-                    ok = wait_bar(bar(C::kBarDqFree), ph, abort_flag);
+                    // without dQ^T the dP^T columns are free once dS(i) is in place
+                    ok = !with_dq || wait_bar(bar(C::kBarDqFree), ph, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     {
@@ -587,7 +598,7 @@ __global__ void __launch_bounds__(512, 1)
             const int dcol = (D == 128) ? wq * 32 + lane : wq * 16 + (lane & 15);
             QIter<BM, GENERAL> it;
             int i;
-            while (it.next(p, j, i)) {
+            while (p.dqacc != nullptr && it.next(p, j, i)) {
                 ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();

@@ -252,12 +252,15 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             issue_dvdk(s, pb, cnt > 0);
             __syncwarp();
-            ok = wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
+            const bool with_dq = p.dqacc != nullptr;   // else the deterministic dQ pass computes dQ
+            ok = !with_dq || wait_bar(bar(C::kBarDqEmpty), (cnt & 1) ^ 1u, abort_flag);
             if (!ok) break;
             tc_fence_after();
             {
-                issue_dq(pb);
-                mma_commit(bar(C::kBarDqFull), leader);
+                if (with_dq) {
+                    issue_dq(pb);
+                    mma_commit(bar(C::kBarDqFull), leader);
+                }
                 mma_commit(bar(C::kBarPdsEmpty + pb), leader);
                 mma_commit(bar(C::kBarQEmpty + s), leader);
             }
@@ -380,6 +383,10 @@ __global__ void __launch_bounds__(320, 1)
         QIter<BM, GENERAL> it;
         int i;
         while (it.next(p, j, i)) {
+            if (p.dqacc == nullptr) {   // no dQ: only count the tiles (the dK epilogue needs cnt)
+                ++cnt;
+                continue;
+            }
             ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();

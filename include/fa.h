@@ -155,6 +155,30 @@ FA_API int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
                      int window_left, int window_right, const float *alibi_slopes,
                      const uint8_t *block_mask, int dtype, void *stream);
 
+/*
+ * Bytes of device workspace fa_bwd_deterministic needs: the two fp32 per-row
+ * statistics [B][H][Npad] only (no dQ accumulator).  0 for invalid sizes.
+ */
+FA_API size_t fa_bwd_deterministic_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+
+/*
+ * Deterministic backward: the arguments, layouts and results of fa_bwd_ex,
+ * with every output bitwise reproducible from run to run ("深度解析"
+ * section 五 notes that a fully deterministic backward costs speed).  dK and
+ * dV come from the key-block kernel as in fa_bwd_ex (same bits); dQ comes
+ * from a second sweep, one CTA per 128 query rows, that recomputes S and dP
+ * and sums dS K over the visible key blocks in increasing order in tensor
+ * memory -- no atomics.  It performs seven matrix products per visible
+ * block pair instead of five.  workspace: at least
+ * fa_bwd_deterministic_workspace_bytes() bytes, 16-byte aligned.
+ */
+FA_API int fa_bwd_deterministic(const void *q, const void *k, const void *v, const void *o,
+                                const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                                void *workspace, size_t workspace_bytes,
+                                int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                                int window_left, int window_right, const float *alibi_slopes,
+                                const uint8_t *block_mask, int dtype, void *stream);
+
 /* Block-sparse backward; block_mask as for fa_fwd_blocksparse. */
 FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
                               const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -218,11 +242,12 @@ FA_API int fa_last_timeout_site(int *site);
  * launches.  fa_profile_read() waits for those events, writes the summed
  * milliseconds and launch counts per kernel kind, clears the record and
  * returns FA_OK.  Kinds: 0 forward, 1 backward pre-pass (D and accumulator
- * reset), 2 backward main kernel, 3 backward dQ conversion.  ms and launches
+ * reset), 2 backward main kernel, 3 backward dQ conversion, 4 dQ pass of the
+ * deterministic backward.  ms and launches
  * are HOST arrays of FA_PROFILE_KINDS entries.  Events are created and
  * destroyed by the library; no device memory is allocated.
  */
-#define FA_PROFILE_KINDS 4
+#define FA_PROFILE_KINDS 5
 FA_API int fa_profile_enable(int on);
 FA_API int fa_profile_read(float *ms, int *launches);
 

@@ -104,6 +104,26 @@ def test_bwd_rejects():
     assert _bwd(mask=NULL) == INVALID
 
 
+def test_deterministic_workspace_and_rejects():
+    lib = fa.load_library()
+    B, H, Nq, Nk, d = 2, 3, 1000, 700, 256
+    npad = (Nq + 127) // 128 * 128          # two per-row statistics, no dQ accumulator
+    assert lib.fa_bwd_deterministic_workspace_bytes(B, H, Nq, Nk, d) == 2 * B * H * npad * 4
+    assert lib.fa_bwd_deterministic_workspace_bytes(1, 1, 1, 0, 64) == 0
+    assert lib.fa_bwd_deterministic_workspace_bytes(1, 1, 1, 1, 96) == 0
+    need = lib.fa_bwd_deterministic_workspace_bytes(1, 1, 128, 128, 64)
+
+    def det(ws=A, ws_bytes=need, d=64, dq=A, scale=0.125):
+        return lib.fa_bwd_deterministic(A, A, A, A, A, A, dq, A, A, ws, ws_bytes, 1, 1, 128, 128, d, scale, 0,
+                                        -1, -1, NULL, NULL, 1, S)
+    assert det(ws=NULL) == WORKSPACE
+    assert det(ws_bytes=need - 1) == WORKSPACE
+    assert det(ws=M) == MISALIGNED
+    assert det(dq=NULL) == INVALID
+    assert det(d=80) == UNSUPPORTED
+    assert det(scale=0.0) == INVALID
+
+
 def test_profile_read_rejects_null():
     lib = fa.load_library()
     assert lib.fa_profile_read(None, None) == INVALID
