@@ -56,6 +56,9 @@ WORKLOADS = {
                       window=(1024, 0)),
     "cross128": dict(B=4, H=16, N=1024, Nk=8192, d=128, dtype="bf16", causal=True, sparse=False, bwd=True),
     "alibi128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True, alibi=True),
+    # the deterministic backward (fa_bwd_deterministic) on the d = 128 sweep's shape
+    "det128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True,
+                   deterministic=True),
 }
 
 
@@ -107,6 +110,7 @@ def describe(name, w):
     s += f" window={w['window']}" if "window" in w else ""
     s += " alibi" if w.get("alibi") else ""
     s += " fwd+bwd" if w["bwd"] else " fwd"
+    s += " (deterministic backward)" if w.get("deterministic") else ""
     return s
 
 
@@ -214,7 +218,8 @@ def make_inputs(w, seed, device):
         import flash_fwd_b200 as fa
         dev["dq"] = torch.empty_like(dev["q"])
         dev["dk"], dev["dv"] = torch.empty_like(dev["k"]), torch.empty_like(dev["v"])
-        dev["ws"] = torch.empty(fa.fa_bwd_ex_workspace_bytes(w["B"], w["H"], w["N"], w.get("Nk", w["N"]), w["d"]),
+        ws_fn = fa.fa_bwd_deterministic_workspace_bytes if w.get("deterministic") else fa.fa_bwd_ex_workspace_bytes
+        dev["ws"] = torch.empty(ws_fn(w["B"], w["H"], w["N"], w.get("Nk", w["N"]), w["d"]),
                                 dtype=torch.uint8, device=device)
     return host, dev
 
@@ -222,7 +227,12 @@ def make_inputs(w, seed, device):
 def step(w, t, stream):
     import flash_fwd_b200 as fa
     scale = 1.0 / w["d"] ** 0.5
-    if general(w):
+    if w.get("deterministic"):
+        fa.fa_fwd_ex(t["q"], t["k"], t["v"], t["o"], t["lse"], w["causal"], scale, w.get("window"), t["slopes"],
+                     t["mask"], stream)
+        fa.fa_bwd_deterministic(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"],
+                                t["ws"], w["causal"], scale, w.get("window"), t["slopes"], t["mask"], stream)
+    elif general(w):
         fa.fa_fwd_ex(t["q"], t["k"], t["v"], t["o"], t["lse"], w["causal"], scale, w.get("window"), t["slopes"],
                      t["mask"], stream)
         if w["bwd"]:
@@ -377,8 +387,12 @@ def run_ours(args, w, name):
     capped = power_capped(clocks)
     peak = sustained if capped and sustained else burst
     peak_kind = "sustained (power-capped run)" if capped and sustained else "burst"
-    if dom in ("fwd", "bwd_main"):
-        alg = fwd_f if dom == "fwd" else bwd_f
+    if dom in ("fwd", "bwd_main", "bwd_dq"):
+        # tensor FLOPs the kernel performs: the backward's five products, of
+        # which the deterministic backward's key-block kernel does four (no dQ)
+        # and its dQ pass three (S and dP again, then dQ)
+        det = w.get("deterministic", False)
+        alg = {"fwd": fwd_f, "bwd_main": bwd_f * (0.8 if det else 1.0), "bwd_dq": bwd_f * 0.6}[dom]
         achieved = alg / (per_launch_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_source": f"{src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
@@ -394,7 +408,7 @@ def run_ours(args, w, name):
              "fwd_frac_of_peak": (fwd_f / (fwd_ms / 1e3) / 1e12) / peak if fwd_ms else None,
              "peak": peak, "peak_kind": peak_kind}
     if w["bwd"]:
-        bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post")) / max(prof["bwd_main"][1], 1)
+        bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post", "bwd_dq")) / max(prof["bwd_main"][1], 1)
         split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12
         split["bwd_frac_of_peak"] = split["bwd_tflops"] / peak
 
