@@ -123,8 +123,8 @@ int check_problem(const Problem &pr) {
 }
 
 template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
-int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const fa::FwdParams &p,
-               int BH, cudaStream_t stream) {
+int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mo,
+               const fa::FwdParams &p, int BH, cudaStream_t stream) {
     using C = fa::FwdCfg<D, NQ, NSK, NSV>;
     auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, GENERAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
@@ -133,17 +133,17 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     if (ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(ctas));
     ProfScope prof(0, stream);
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <bool BF16, bool GENERAL>
-int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mo,
                  const fa::FwdParams &p, int BH, cudaStream_t s) {
     switch (d) {
-        case 64: return launch_fwd<64, 2, 6, 4, BF16, GENERAL>(mq, mk, mv, p, BH, s);
-        case 128: return launch_fwd<128, 2, 3, 2, BF16, GENERAL>(mq, mk, mv, p, BH, s);
-        case 256: return launch_fwd<256, 1, 1, 1, BF16, GENERAL>(mq, mk, mv, p, BH, s);
+        case 64: return launch_fwd<64, 2, 6, 4, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
+        case 128: return launch_fwd<128, 2, 3, 2, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, 1, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
         default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -156,12 +156,12 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
         return FA_ERR_MISALIGNED;
     const int BH = static_cast<int>(pr.BH());
     if (static_cast<long long>(BH) * ((pr.Nq + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // 1-D grid
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if ((rc = make_map(&mq, q, pr.d, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mo, o, pr.d, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mk, k, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mv, v, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     fa::FwdParams p;
-    p.o = o;
     p.lse = lse;
     p.mask = pr.mask;
     p.alibi = pr.alibi;
@@ -180,10 +180,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool general = pr.general();
     if (pr.dtype == FA_BF16)
-        return general ? dispatch_fwd<true, true>(pr.d, mq, mk, mv, p, BH, s)
-                       : dispatch_fwd<true, false>(pr.d, mq, mk, mv, p, BH, s);
-    return general ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, p, BH, s)
-                   : dispatch_fwd<false, false>(pr.d, mq, mk, mv, p, BH, s);
+        return general ? dispatch_fwd<true, true>(pr.d, mq, mk, mv, mo, p, BH, s)
+                       : dispatch_fwd<true, false>(pr.d, mq, mk, mv, mo, p, BH, s);
+    return general ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, mo, p, BH, s)
+                   : dispatch_fwd<false, false>(pr.d, mq, mk, mv, mo, p, BH, s);
 }
 
 

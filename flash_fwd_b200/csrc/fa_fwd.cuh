@@ -46,7 +46,6 @@ namespace fa {
 enum MaskMode : int { kDense = 0, kCausal = 1, kSparse = 2 };
 
 struct FwdParams {
-    void *o;                  // [BH][Nq][D] 16-bit
     float *lse;               // [BH][Nq]
     const uint8_t *mask;      // [nqb][nkb] block mask (kSparse)
     const float *alibi;       // [H] ALiBi slopes (natural-log units of the score) or null (GENERAL kernels)
@@ -161,7 +160,7 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
 template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-               const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, const FwdParams p) {
     using C = FwdCfg<D, NQ, NSK, NSV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -208,6 +207,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmo);
     }
     tc_fence_before();
     __syncthreads();
@@ -504,12 +504,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         }
         if (ok && cnt > 0) ok = wait_bar(bar(C::kBarOFull + t), 0, abort_flag);
         tc_fence_after();
-        if (rb < p.nqb && ok) {
+        // O_t is staged in the Q_t buffer (every S product has completed once
+        // O_t is final) as 128-byte-swizzled 64-column chunks, then written by
+        // TMA stores: one thread per row would touch 32 lines per store
+        const bool epi = rb < p.nqb && ok;
+        uint8_t *stage = smem + C::kQOff + t * C::kTileBytes;
+        if (epi) {
             const bool valid = row < p.Nq;
             const float l_o = BF16 ? l_r : l;
             const float inv_l = (cnt > 0 && l_o > 0.f) ? 1.0f / l_o : 0.0f;
-            uint8_t *orow = reinterpret_cast<uint8_t *>(p.o) +
-                            (static_cast<size_t>(bh) * p.Nq + (valid ? row : 0)) * D * 2;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -525,11 +528,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 for (int k = 0; k < 16; ++k)
                     pk[k] = pack2<BF16>(__uint_as_float(o[2 * k]) * inv_l,
                                         __uint_as_float(o[2 * k + 1]) * inv_l);
-                if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 64);
+                uint8_t *srow = stage + (q >> 1) * C::kChunkBytes + row_local * 128;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                for (int k = 0; k < 4; ++k) {
+                    const int u = (q & 1) * 4 + k;   // 16-byte unit within the 128-byte row
+                    *reinterpret_cast<uint4 *>(srow + ((u ^ (row_local & 7)) << 4)) =
+                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                 }
             }
             if (valid) {
@@ -537,6 +541,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                                                         : -INFINITY;
                 p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
             }
+        }
+        fence_async_smem();
+        named_sync(1 + t, 128);   // the four warps of query tile t (every one of them gets here)
+        if (epi && wq == 0 && lane == 0) {
+            for (int c = 0; c < C::kChunks; ++c)
+                tma_store_3d(&tmo, smem_u32(stage + c * C::kChunkBytes), c * 64, rb * 128, bh);   // rows >= Nq clipped
+            bulk_commit();
+            bulk_wait_read();   // shared memory stays allocated until the stores have read it
         }
     }
 
