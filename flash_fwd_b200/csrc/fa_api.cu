@@ -228,6 +228,8 @@ int launch_bwd_dq(const BwdBuffers &bb, const Problem &pr, fa::BwdParams p, cons
     int rc;
     if ((rc = make_map(&mq, bb.q, D, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mdo, bb.dout, D, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
+    CUtensorMap mdq;
+    if ((rc = make_map(&mdq, bb.dq, D, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
     p.nqt = (pr.Nq + 127) / 128;
     p.dq = bb.dq;
     auto kern = fa::bwd_dq_kernel<D, BF16, GENERAL>;
@@ -235,7 +237,7 @@ int launch_bwd_dq(const BwdBuffers &bb, const Problem &pr, fa::BwdParams p, cons
         return FA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nqt));
     ProfScope prof(4, stream);
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -252,8 +254,10 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuf
     float *dqacc = deterministic ? nullptr : dvec + static_cast<size_t>(BH) * Npad;
     int rc = launch_bwd_pre<D, BF16>(bb.o, bb.dout, bb.lse, lse2, dvec, dqacc, BH, pr.Nq, Npad, stream);
     if (rc != FA_OK) return rc;
-    CUtensorMap mk, mv, mq, mdo;
+    CUtensorMap mk, mv, mq, mdo, mdk, mdv;
     if ((rc = make_map(&mk, bb.k, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mdk, bb.dk, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map(&mdv, bb.dv, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mv, bb.v, D, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mq, bb.q, D, pr.Nq, BH, pr.dtype, BM)) != FA_OK) return rc;
     if ((rc = make_map(&mdo, bb.dout, D, pr.Nq, BH, pr.dtype, BM)) != FA_OK) return rc;
@@ -285,7 +289,7 @@ int launch_bwd(Kernel kern, int smem_bytes, int threads, int split, const BwdBuf
         // one-dimensional grid of BH x key blocks (x split) CTAs
         const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb * split));
         ProfScope prof(2, stream);
-        kern<<<grid, threads, smem_bytes, stream>>>(mk, mv, mq, mdo, p);
+        kern<<<grid, threads, smem_bytes, stream>>>(mk, mv, mq, mdo, mdk, mdv, p);
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (deterministic) return launch_bwd_dq<D, BF16, GENERAL>(bb, pr, p, mk, mv, stream);

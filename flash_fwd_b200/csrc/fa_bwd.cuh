@@ -235,6 +235,7 @@ template <int D, int NS, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
+               const __grid_constant__ CUtensorMap tmdk, const __grid_constant__ CUtensorMap tmdv,
                const BwdParams p) {
     using C = BwdCfg<D, NS>;
     constexpr int BM = C::BM;
@@ -555,15 +556,17 @@ __global__ void __launch_bounds__(512, 1)
             }
             // ------------------------------------------------------------ dV / dK epilogue
             {
+                // dV (warps 0-3) and dK (warps 4-7) are staged as 128-byte-swizzled
+                // 64-column chunks in the V_j / K_j buffers (free once every
+                // product has completed) and written by TMA stores
                 bool done = ok;
                 if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
                 tc_fence_after();
                 const bool is_dv = warp < 4;
                 const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
                 const int r = (warp & 3) * 32 + lane;
-                const int key = j * 128 + r;
                 const float mul = is_dv ? 1.0f : p.scale;
-                uint8_t *out = reinterpret_cast<uint8_t *>(is_dv ? p.dv : p.dk);
+                uint8_t *stage = smem + (is_dv ? C::kVOff : C::kKOff);
                 const uint32_t col0 = is_dv ? C::kColDV : C::kColDK;
                 if (done) {
         #pragma unroll 1
@@ -574,18 +577,28 @@ __global__ void __launch_bounds__(512, 1)
                             tmem_ld_wait();
                         } else {
     #pragma unroll
-                            for (int k = 0; k < 32; ++k) v[k] = 0u;
+                            for (int k = 0; k < 32; ++k) v[k] = 0u;   // no query sees this key block
                         }
-                        if (key < p.Nk) {
-                            uint32_t pk[16];
+                        uint32_t pk[16];
     #pragma unroll
-                            for (int k = 0; k < 16; ++k)
-                                pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-                            uint4 *dst = reinterpret_cast<uint4 *>(out + ((static_cast<size_t>(bh) * p.Nk + key) * D + 32 * ch) * 2);
+                        for (int k = 0; k < 16; ++k)
+                            pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+                        uint8_t *srow = stage + (ch >> 1) * C::kChunk + r * 128;
     #pragma unroll
-                            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                        for (int k = 0; k < 4; ++k) {
+                            const int u = (ch & 1) * 4 + k;
+                            *reinterpret_cast<uint4 *>(srow + ((u ^ (r & 7)) << 4)) =
+                                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                         }
                     }
+                }
+                fence_async_smem();
+                named_sync(is_dv ? 1 : 2, 128);   // the four warps of this output (every one gets here)
+                if (done && (warp & 3) == 0 && lane == 0) {
+                    for (int c = 0; c < D / 64; ++c)   // keys >= Nk are clipped
+                        tma_store_3d(is_dv ? &tmdv : &tmdk, smem_u32(stage + c * C::kChunk), c * 64, j * 128, bh);
+                    bulk_commit();
+                    bulk_wait_read();
                 }
             }
         } else {

@@ -121,7 +121,7 @@ template <int D, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdq, const BwdParams p) {
     using C = DqCfg<D>;
     constexpr int NSK = C::NSK;
     constexpr int NSV = C::NSV;
@@ -484,11 +484,13 @@ __global__ void __launch_bounds__(352, 1)
             ++cnt;
         }
         // ------------------------------------------------------------ dQ epilogue
+        // staged as 128-byte-swizzled 64-column chunks in the Q_i buffer (free
+        // once every product has completed), written by TMA stores
         bool done = ok;
         if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
         tc_fence_after();
         if (done) {
-            // this thread: row q, d columns [kh D / 2, (kh + 1) D / 2)
+            // this thread: row `row`, d columns [kh D / 2, (kh + 1) D / 2)
 #pragma unroll 1
             for (int ch = 0; ch < D / 64; ++ch) {
                 uint32_t v[32];
@@ -499,17 +501,27 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] = 0u;   // a tile that sees no key: dQ = 0
                 }
-                if (q < p.Nq) {
-                    uint32_t pk[16];
+                uint32_t pk[16];
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * p.scale, __uint_as_float(v[2 * k + 1]) * p.scale);
-                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(p.dq) +
-                                                           ((static_cast<size_t>(bh) * p.Nq + q) * D + kh * (D / 2) + 32 * ch) * 2);
+                for (int k = 0; k < 16; ++k)
+                    pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * p.scale, __uint_as_float(v[2 * k + 1]) * p.scale);
+                const int col = kh * (D / 2) + 32 * ch;
+                uint8_t *srow = smem + C::kQOff + (col / 64) * C::kChunk + row * 128;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                for (int k = 0; k < 4; ++k) {
+                    const int u = (col % 64) / 8 + k;
+                    *reinterpret_cast<uint4 *>(srow + ((u ^ (row & 7)) << 4)) =
+                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                 }
             }
+        }
+        fence_async_smem();
+        named_sync(1, 256);   // the eight softmax-grad warps (every one gets here)
+        if (done && warp == 0 && lane == 0) {
+            for (int c = 0; c < D / 64; ++c)   // rows >= Nq are clipped
+                tma_store_3d(&tmdq, smem_u32(smem + C::kQOff + c * C::kChunk), c * 64, i * 128, bh);
+            bulk_commit();
+            bulk_wait_read();
         }
     }
 
