@@ -79,6 +79,27 @@ int oracle_bwd_dkdv_cols(const double *q, const double *k, const double *v, cons
                          const uint8_t *mask, int blk, const int *cols, int ncols,
                          double *dk, double *dv, int nthreads);
 
+/*
+ * FP8 (E4M3) forward with block quantisation and incoherent processing (the
+ * readings are written out above the FP8 section of oracle.c).
+ *   oracle_e4m3_value / _round: decode a code; round a value to a code.
+ *   oracle_rotate_f32: x [nrows][d] <- (x o signs) H_d / sqrt(d) in float.
+ *   oracle_fp8_quantize: x float [BH][N][d] -> codes [BH][N][d] and scales
+ *     [BH][ceil(N/rows)] (rows per block), rotating first when signs != NULL.
+ *   oracle_fwd_fp8: O [BH][nrows][d], LSE [BH][nrows] on query rows qrows from
+ *     the codes and scales (sq, sk [BH][ceil(N/rows)], sv [BH]); quant_p = 0
+ *     keeps P unrounded.
+ */
+double oracle_e4m3_value(int code);
+int oracle_e4m3_round(double x);
+int oracle_e4m3_round_array(const double *x, long n, uint8_t *codes);
+int oracle_rotate_f32(float *x, long nrows, int d, const float *signs);
+int oracle_fp8_quantize(const float *x, int BH, int N, int d, int rows, const float *signs,
+                        uint8_t *codes, float *scales);
+int oracle_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, const float *sq, const float *sk,
+                   const float *sv, int BH, int N, int d, int rows, double scale, int causal, int quant_p,
+                   const int *qrows, int nrows, double *o, double *lse, int nthreads);
+
 #ifdef __cplusplus
 }
 #endif

@@ -58,8 +58,17 @@ def _lib():
         lib.oracle_bwd_full_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, D, D, D, D, D, i]
         lib.oracle_bwd_dq_rows_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, I32, i, D, i]
         lib.oracle_bwd_dkdv_cols_ex.argtypes = [D, D, D, D, i, i, i, i, i, f, i, i, i, D, U8, i, I32, i, D, D, i]
+        F32 = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_e4m3_value.argtypes = [i]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_round.argtypes = [f]
+        lib.oracle_e4m3_round_array.argtypes = [D, ctypes.c_long, U8]
+        lib.oracle_rotate_f32.argtypes = [F32, ctypes.c_long, i, F32]
+        lib.oracle_fp8_quantize.argtypes = [F32, i, i, i, i, F32, U8, F32]
+        lib.oracle_fwd_fp8.argtypes = [U8, U8, U8, F32, F32, F32, i, i, i, i, f, i, i, I32, i, D, D, i]
         for fn in (lib.oracle_fwd_rows_ex, lib.oracle_online_softmax_fwd_ex, lib.oracle_bwd_full_ex,
-                   lib.oracle_bwd_dq_rows_ex, lib.oracle_bwd_dkdv_cols_ex):
+                   lib.oracle_bwd_dq_rows_ex, lib.oracle_bwd_dkdv_cols_ex, lib.oracle_e4m3_round,
+                   lib.oracle_e4m3_round_array, lib.oracle_rotate_f32, lib.oracle_fp8_quantize, lib.oracle_fwd_fp8):
             fn.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -202,3 +211,72 @@ def bwd_dkdv_cols(q, k, v, dout, scale, cols, flags=0, mask=None, blk=128, nthre
                                         _dp(dk), _dp(dv), _threads(nthreads))
     assert rc == 0, rc
     return dk, dv
+
+
+# --------------------------------------------------------------------------
+# FP8 forward (block quantisation + incoherent processing); the readings are
+# written out above the FP8 section of oracle.c
+# --------------------------------------------------------------------------
+def _u8p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+
+
+def _f32p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def e4m3_values():
+    """float64 [256]: the value of every E4M3 code (NaN for the two NaN codes)."""
+    return np.array([_lib().oracle_e4m3_value(c) for c in range(256)])
+
+
+def e4m3_round(x):
+    """uint8 codes of the values x (nearest, ties to even, saturating at 448)."""
+    x = _f64(x)
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    rc = _lib().oracle_e4m3_round_array(_dp(x), x.size, _u8p(codes))
+    assert rc == 0, rc
+    return codes
+
+
+def rotate_f32(x, signs):
+    """float32 rows x [..., d] <- (x o signs) H_d / sqrt(d), in float."""
+    x = np.ascontiguousarray(np.array(x, dtype=np.float32))
+    s = np.ascontiguousarray(np.asarray(signs, dtype=np.float32))
+    d = x.shape[-1]
+    rc = _lib().oracle_rotate_f32(_f32p(x), x.size // d, d, _f32p(s))
+    assert rc == 0, rc
+    return x
+
+
+def fp8_quantize(x, rows, signs=None):
+    """x [BH, N, d] (float32) -> (codes uint8 [BH, N, d], scales float32 [BH, ceil(N / rows)])."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    if x.ndim == 2:
+        x = x[None]
+    BH, N, d = x.shape
+    nb = (N + rows - 1) // rows
+    codes = np.zeros((BH, N, d), dtype=np.uint8)
+    scales = np.zeros((BH, nb), dtype=np.float32)
+    s = None if signs is None else np.ascontiguousarray(np.asarray(signs, dtype=np.float32))
+    rc = _lib().oracle_fp8_quantize(_f32p(x), BH, N, d, int(rows), None if s is None else _f32p(s),
+                                    _u8p(codes), _f32p(scales))
+    assert rc == 0, rc
+    return codes, scales
+
+
+def fwd_fp8(q8, k8, v8, sq, sk, sv, scale, causal=False, rows=None, quant_p=True, blk=128, nthreads=None):
+    """O [BH, len(rows), d] and LSE [BH, len(rows)] of FP8 attention on the codes
+    (q8, k8, v8 uint8 [BH, N, d]) and scales (sq, sk [BH, ceil(N / blk)], sv [BH])."""
+    q8, k8, v8 = (np.ascontiguousarray(np.asarray(t, dtype=np.uint8)) for t in (q8, k8, v8))
+    sq, sk, sv = (np.ascontiguousarray(np.asarray(t, dtype=np.float32)) for t in (sq, sk, sv))
+    BH, N, d = q8.shape
+    rows = np.arange(N, dtype=np.int32) if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    o = np.zeros((BH, len(rows), d))
+    lse = np.zeros((BH, len(rows)))
+    rc = _lib().oracle_fwd_fp8(_u8p(q8), _u8p(k8), _u8p(v8), _f32p(sq), _f32p(sk), _f32p(sv), BH, N, d, int(blk),
+                               float(scale), int(bool(causal)), int(bool(quant_p)),
+                               rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), len(rows), _dp(o), _dp(lse),
+                               _threads(nthreads))
+    assert rc == 0, rc
+    return o, lse

@@ -1,0 +1,193 @@
+"""Pins of the oracle's FP8 forward ("FlashAttention 深度解析" section 四: FP8
+block quantisation with incoherent processing) against what the format
+definition, the mathematics and independent library routines fix:
+
+* E4M3 decoding at the format's landmark codes, encoding as the exact inverse
+  on every finite code, ties to even, saturation, and agreement with
+  PyTorch's float8_e4m3fn conversion on in-range values;
+* the rotation equals the explicit Sylvester Hadamard matrix (scipy) with the
+  sign flips, is orthogonal (preserves Q K^T), and is its own inverse up to
+  the signs;
+* the quantiser maps every block's largest magnitude to 448 exactly and every
+  value to within half an E4M3 step;
+* FP8 attention reduces to the exact oracle when the operands are E4M3 values
+  and P is not rounded, returns V exactly for identical V rows and for a row
+  with one visible key, and keeps LSE of the dequantised scores;
+* incoherent processing lowers the error against exact attention on inputs
+  with outlier channels (the page's claim is 2.6x).
+"""
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def test_e4m3_landmark_codes():
+    v = oracle.e4m3_values()
+    assert v[0x00] == 0.0 and np.signbit(v[0x80])
+    assert v[0x01] == 2.0 ** -9                    # smallest subnormal
+    assert v[0x07] == 7 * 2.0 ** -9                # largest subnormal
+    assert v[0x08] == 2.0 ** -6                    # smallest normal
+    assert v[0x38] == 1.0 and v[0xB8] == -1.0      # exponent field 7 = bias
+    assert v[0x7E] == 448.0 and v[0xFE] == -448.0  # 1.75 * 2^8
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    finite = v[[c for c in range(0x7F)]]
+    assert np.all(np.diff(finite) > 0)             # codes 0..0x7e increase
+
+
+def test_e4m3_round_inverts_every_finite_code():
+    v = oracle.e4m3_values()
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)])
+    assert np.array_equal(oracle.e4m3_round(v[codes]), codes.astype(np.uint8))
+
+
+def test_e4m3_round_ties_and_saturation():
+    r = lambda x: int(oracle.e4m3_round([x])[0])   # noqa: E731
+    assert r(1 + 2 ** -4) == 0x38                  # tie between 1 and 1.125 -> even mantissa
+    assert r(1 + 3 * 2 ** -4) == 0x3A              # tie between 1.125 and 1.25 -> 1.25
+    assert r(2 ** -10) == 0x00 and r(3 * 2 ** -10) == 0x02   # subnormal ties
+    assert r(1 + 2 ** -4 + 1e-9) == 0x39           # just above the tie
+    for x in (448.0, 449.0, 470.0, 1e30):
+        assert r(x) == 0x7E and r(-x) == 0xFE
+    assert r(float("nan")) == 0x7F
+
+
+def test_e4m3_round_matches_torch_float8():
+    g = np.random.default_rng(0)
+    x = np.concatenate([g.normal(0, 1, 20000), g.normal(0, 50, 20000), g.uniform(-448, 448, 20000),
+                        g.normal(0, 2 ** -7, 20000)]).astype(np.float32).astype(np.float64)
+    ours = oracle.e4m3_round(x)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_rotation_is_the_signed_hadamard_matrix(d):
+    g = np.random.default_rng(d)
+    signs = g.choice([-1.0, 1.0], d)
+    x = g.normal(0, 1, (40, d)).astype(np.float32)
+    got = oracle.rotate_f32(x, signs).astype(np.float64)
+    want = (x.astype(np.float64) * signs) @ scipy.linalg.hadamard(d) / np.sqrt(d)
+    assert np.abs(got - want).max() <= 1e-5 * np.abs(want).max()
+    # orthogonal: dot products (hence Q K^T) are preserved
+    y = g.normal(0, 1, (40, d)).astype(np.float32)
+    ry = oracle.rotate_f32(y, signs).astype(np.float64)
+    assert np.allclose(got @ ry.T, x.astype(np.float64) @ y.astype(np.float64).T, atol=1e-4)
+    # H H = d I: rotating twice with unit signs gives x back (signs flip once more)
+    back = oracle.rotate_f32(oracle.rotate_f32(x, signs), np.ones(d))
+    assert np.abs(back * signs - x).max() <= 1e-5 * np.abs(x).max()
+
+
+def test_quantize_blocks():
+    g = np.random.default_rng(1)
+    BH, N, d, rows = 3, 300, 128, 128
+    x = (g.normal(0, 1, (BH, N, d)) * g.uniform(0.01, 10, (BH, N, 1))).astype(np.float32)
+    x[1, 128:256] = 0.0                                 # an all-zero block
+    codes, scales = oracle.fp8_quantize(x, rows)
+    v = oracle.e4m3_values()
+    assert scales.shape == (BH, 3)
+    assert scales[1, 1] == 1.0 and not codes[1, 128:256].any()
+    for h in range(BH):
+        for b in range(3):
+            blk = x[h, b * rows:(b + 1) * rows]
+            cb = codes[h, b * rows:(b + 1) * rows]
+            if not blk.any():
+                continue
+            amax = np.abs(blk).max()
+            assert scales[h, b] == np.float32(amax) / np.float32(448.0)
+            assert np.abs(v[cb]).max() == 448.0        # the largest magnitude maps to 448
+            y = blk.astype(np.float64) * float(np.float32(448.0) / np.float32(amax))
+            err = np.abs(v[cb] - y)
+            # within half a step: 2^-4 relative for normals, 2^-10 absolute below 2^-6
+            assert np.all(err <= np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-12))
+
+
+def test_quantize_with_rotation_is_rotation_then_quantize():
+    g = np.random.default_rng(2)
+    d = 128
+    signs = g.choice([-1.0, 1.0], d)
+    x = g.normal(0, 1, (2, 200, d)).astype(np.float32)
+    c1, s1 = oracle.fp8_quantize(x, 128, signs)
+    c2, s2 = oracle.fp8_quantize(oracle.rotate_f32(x, signs), 128)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def _codes_and_values(g, shape, scale=1.0):
+    """Random E4M3 codes (no NaN) of values around `scale`, and their values."""
+    v = oracle.e4m3_values()
+    pool = np.array([c for c in range(256) if c not in (0x7F, 0xFF) and abs(v[c]) <= 8 * scale + 1e-12])
+    codes = g.choice(pool, size=shape).astype(np.uint8)
+    return codes, v[codes]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_attention_reduces_to_exact_oracle(causal):
+    g = np.random.default_rng(3)
+    BH, N, d = 2, 200, 64
+    q8, qv = _codes_and_values(g, (BH, N, d))
+    k8, kv = _codes_and_values(g, (BH, N, d))
+    v8, vv = _codes_and_values(g, (BH, N, d))
+    sq = g.uniform(0.01, 0.05, (BH, 2)).astype(np.float32)
+    sk = g.uniform(0.01, 0.05, (BH, 2)).astype(np.float32)
+    sv = g.uniform(0.5, 2, BH).astype(np.float32)
+    o, lse = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv, 0.125, causal=causal, quant_p=False)
+    # the same attention on the dequantised operands through the pinned oracle
+    blk = np.arange(N) // 128
+    Q = qv * sq[:, blk][:, :, None]
+    K = kv * sk[:, blk][:, :, None]
+    V = vv * sv[:, None, None]
+    ro, rl = oracle.fwd(Q, K, V, 0.125, oracle.CAUSAL if causal else 0)
+    assert np.allclose(o, ro, rtol=1e-10, atol=1e-12)
+    assert np.allclose(lse, rl, rtol=1e-12, atol=1e-12)
+    # rounding P changes O by a bounded amount and LSE not at all
+    o8, lse8 = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv, 0.125, causal=causal)
+    assert np.array_equal(lse8, lse)
+    assert 0 < np.abs(o8 - o).max() <= 2.0 ** -3 * np.abs(V).max()
+
+
+def test_fp8_attention_exact_cases():
+    g = np.random.default_rng(4)
+    BH, N, d = 1, 150, 64
+    q8, _ = _codes_and_values(g, (BH, N, d))
+    k8, _ = _codes_and_values(g, (BH, N, d))
+    v8 = np.repeat(_codes_and_values(g, (BH, 1, d))[0], N, axis=1)   # identical V rows
+    vals = oracle.e4m3_values()
+    sq = sk = np.full((BH, 2), 0.03, np.float32)
+    sv = np.full(BH, 1.5, np.float32)
+    o, _ = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv, 0.2, causal=True)
+    assert np.allclose(o, np.broadcast_to(vals[v8[0, 0]] * 1.5, o.shape), rtol=1e-12, atol=0)
+    # causal row 0 sees key 0 only
+    v8 = _codes_and_values(g, (BH, N, d))[0]
+    o, _ = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv, 0.2, causal=True, rows=[0])
+    assert np.allclose(o[0, 0], vals[v8[0, 0]] * 1.5, rtol=1e-12, atol=0)
+
+
+def _exact(q, k, v, scale):
+    s = scale * q @ k.transpose(0, 2, 1)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    return (p / p.sum(-1, keepdims=True)) @ v
+
+
+def test_incoherent_processing_lowers_the_error():
+    # Q and K with a few outlier channels (the case incoherent processing targets)
+    g = np.random.default_rng(5)
+    BH, N, d = 2, 256, 128
+    q = g.normal(0, 1, (BH, N, d))
+    k = g.normal(0, 1, (BH, N, d))
+    q[..., :4] *= 30.0
+    k[..., :4] *= 30.0
+    v = g.normal(0, 1, (BH, N, d))
+    scale = 0.5 / np.sqrt(d)
+    ref = _exact(q, k, v, scale)
+    v8, sv = oracle.fp8_quantize(v.astype(np.float32), N)
+    errs = {}
+    for name, signs in (("plain", None), ("incoherent", g.choice([-1.0, 1.0], d))):
+        q8, sq = oracle.fp8_quantize(q.astype(np.float32), 128, signs)
+        k8, sk = oracle.fp8_quantize(k.astype(np.float32), 128, signs)
+        o, _ = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv[:, 0], scale)
+        errs[name] = np.sqrt(np.mean((o - ref) ** 2))
+    assert errs["incoherent"] * 1.5 < errs["plain"], errs

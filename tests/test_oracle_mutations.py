@@ -37,9 +37,25 @@ MUTANTS = {
     "alibi_head_ignored": ("return -sp->slopes[h % sp->H] * dist;", "return -sp->slopes[0] * dist;"),
 }
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+# FP8 forward (E4M3, rotation, block quantiser, FP8 attention): checked by its own pins
+FP8_MUTANTS = {
+    "e4m3_bias_off_by_one": ("else v = ldexp(1.0 + m / 8.0, e - 7);", "else v = ldexp(1.0 + m / 8.0, e - 6);"),
+    "e4m3_ties_to_odd": ("(dd == bd && (c & 1) == 0)", "(dd == bd && (c & 1) == 1)"),
+    "rotation_butterfly_sign": ("x[c + h] = a - b;", "x[c + h] = b - a;"),
+    "quantiser_scale_inverted": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
+                                 "const float inv = amax > 0.0f ? amax / 448.0f : 1.0f;"),
+    "fp8_v_scale_dropped": ("const double f = (double)c->sv[h] / l8;", "const double f = 1.0 / l8;"),
+    "fp8_key_scale_uses_query_block": ("(double)c->sk[h * nb + j / c->rows]", "(double)c->sk[h * nb + i / c->rows]"),
+}
+
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_modes.py"]
+FP8_PIN_FILES = ["test_oracle_fp8.py"]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(FP8_MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
-    old, new = MUTANTS[name]
+    old, new = MUTANTS[name] if name in MUTANTS else FP8_MUTANTS[name]
+    files = PIN_FILES if name in MUTANTS else FP8_PIN_FILES
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor not found for {name}"
     mut = src.replace(old, new)
@@ -50,7 +66,6 @@ def test_pins_catch_mutant(name, tmp_path):
                     "-o", str(lib), str(cfile), "-lm", "-lpthread"], check=True)
     env = dict(os.environ, ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_modes.py")],
+                        *[os.path.join(ROOT, "tests", f) for f in files]],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
