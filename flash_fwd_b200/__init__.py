@@ -16,7 +16,7 @@ __all__ = [
     "fa_bwd_blocksparse", "fa_bwd_workspace_bytes", "fa_status_string", "fa_last_device_status", "fa_last_timeout_site",
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
     "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes", "fa_bwd_deterministic",
-    "fa_bwd_deterministic_workspace_bytes",
+    "fa_bwd_deterministic_workspace_bytes", "fa_fp8_quantize_qkv", "fa_fwd_fp8", "attention_fwd_fp8",
 ]
 
 FA_BLOCK = 128
@@ -60,6 +60,8 @@ def load_library():
     lib.fa_bwd_deterministic_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_bwd_deterministic_workspace_bytes.restype = sz
     lib.fa_bwd_deterministic.argtypes = list(lib.fa_bwd_ex.argtypes)
+    lib.fa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, i, vp]
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -68,7 +70,7 @@ def load_library():
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
-               lib.fa_bwd_deterministic,
+               lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -96,7 +98,7 @@ def fa_version():
     return load_library().fa_version()
 
 
-PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post", "bwd_dq")
+PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post", "bwd_dq", "fp8_quant", "fwd_fp8")
 
 
 def fa_profile_enable(on=True):
@@ -272,3 +274,37 @@ def attention_bwd(q, k, v, o, dout, lse, causal=False, scale=None, block_mask=No
     else:
         fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask, causal, scale, stream)
     return dq, dk, dv
+
+
+def fa_fp8_quantize_qkv(q, k, v, signs=None, stream=None):
+    """E4M3 codes and scales of q, k, v [B, H, N, d] (16-bit, on the device):
+    returns (q8, k8, v8 uint8 [B, H, N, d], sq, sk, sv fp32 [B, H, ceil(N / 128)]).
+    signs (fp32 [d] of +-1 on the device) rotates Q and K by diag(signs) H_d / sqrt(d)."""
+    B, H, N, d = _shape(q)
+    nb = (N + 127) // 128
+    q8, k8, v8 = (torch.empty((B, H, N, d), dtype=torch.uint8, device=q.device) for _ in range(3))
+    sq, sk, sv = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
+    rc = load_library().fa_fp8_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq),
+                                            _ptr(sk), _ptr(sv), B, H, N, d, _ptr(signs), _dtype(q), _stream(stream))
+    _check(rc, "fa_fp8_quantize_qkv")
+    return q8, k8, v8, sq, sk, sv
+
+
+def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal=False, scale=None, stream=None):
+    """FP8 forward on the codes and scales of fa_fp8_quantize_qkv; o [B, H, N, d]
+    (float16 or bfloat16) and lse [B, H, N] fp32 are written."""
+    B, H, N, d = _shape(q8)
+    rc = load_library().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
+                                   B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(o), _stream(stream))
+    _check(rc, "fa_fwd_fp8")
+
+
+def attention_fwd_fp8(q, k, v, causal=False, scale=None, signs=None, stream=None):
+    """Quantises q, k, v to E4M3 (rotating Q and K when signs are given) and runs
+    the FP8 forward; returns (o, lse) with o in q's dtype."""
+    B, H, N, d = _shape(q)
+    q8, k8, v8, sq, sk, sv = fa_fp8_quantize_qkv(q, k, v, signs, stream)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal, scale, stream)
+    return o, lse

@@ -14,6 +14,7 @@
 #include "fa_bwd_dq.cuh"
 #include "fa_bwd_split.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_fp8.cuh"
 
 namespace {
 
@@ -81,6 +82,22 @@ int make_map(CUtensorMap *map, const void *base, int d, int N, long long BH, int
     CUresult r = enc(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                      3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// [BH][N][d] E4M3 codes as a 3-D TMA map {d, N, BH} with d x 128 x 1 boxes
+// (d = 128: one 128-byte swizzle atom per row); rows past N read as zeros.
+int make_map8(CUtensorMap *map, const void *base, int d, int N, long long BH) {
+    auto enc = encode_fn();
+    if (!enc) return FA_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                             static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(d), 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -370,9 +387,114 @@ int noalloc_scratch(void **out) {
     return FA_OK;
 }
 
+// ---------------------------------------------------------------- FP8
+template <int D, bool BF16>
+int launch_quant(const fa::QuantParams &qp, long long BH, cudaStream_t s) {
+    using C = fa::QuantCfg<D>;
+    const long long ctas = BH * qp.nb;
+    if (ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    {
+        ProfScope prof(5, s);
+        fa::fp8_quant_kernel<D, BF16><<<dim3(static_cast<unsigned>(ctas), 3), C::kThreads, 0, s>>>(qp, 0);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    {
+        ProfScope prof(5, s);
+        fa::fp8_quant_kernel<D, BF16><<<dim3(static_cast<unsigned>(ctas), 1), C::kThreads, 0, s>>>(qp, 1);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    {
+        ProfScope prof(5, s);
+        fa::fp8_vscale_kernel<<<static_cast<unsigned>((BH + 255) / 256), 256, 0, s>>>(qp.scales[2], qp.nb, BH);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+FA_API int fa_fp8_quantize_qkv(const void *q, const void *k, const void *v, uint8_t *q8, uint8_t *k8, uint8_t *v8,
+                               float *sq, float *sk, float *sv, int B, int H, int N, int d, const float *signs,
+                               int dtype, void *stream) {
+    if (!q || !k || !v || !q8 || !k8 || !v8 || !sq || !sk || !sv) return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH > 0x7fffffffLL || N > fa::kMaxRows) return FA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q, k, v, q8, k8, v8};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+    const void *fptrs[] = {sq, sk, sv, signs};
+    for (const void *ptr : fptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 3u) return FA_ERR_MISALIGNED;
+    fa::QuantParams qp;
+    qp.src[0] = q;
+    qp.src[1] = k;
+    qp.src[2] = v;
+    qp.dst[0] = q8;
+    qp.dst[1] = k8;
+    qp.dst[2] = v8;
+    qp.scales[0] = sq;
+    qp.scales[1] = sk;
+    qp.scales[2] = sv;
+    qp.signs = signs;
+    qp.rnorm = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    qp.N = N;
+    qp.nb = (N + 127) / 128;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf = dtype == FA_BF16;
+    switch (d) {
+        case 64: return bf ? launch_quant<64, true>(qp, BH, s) : launch_quant<64, false>(qp, BH, s);
+        case 128: return bf ? launch_quant<128, true>(qp, BH, s) : launch_quant<128, false>(qp, BH, s);
+        default: return bf ? launch_quant<256, true>(qp, BH, s) : launch_quant<256, false>(qp, BH, s);
+    }
+}
+
+FA_API int fa_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, const float *sq, const float *sk,
+                      const float *sv, void *o, float *lse, int B, int H, int N, int d, float scale, int causal,
+                      int out_dtype, void *stream) {
+    if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (out_dtype != FA_F16 && out_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    if (N > fa::kMaxRows || BH * ((N + 255) / 256) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q8, k8, v8, o, lse};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+    const void *fptrs[] = {sq, sk, sv};
+    for (const void *ptr : fptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 3u) return FA_ERR_MISALIGNED;
+    CUtensorMap mq, mk, mv, mo;
+    int rc;
+    if ((rc = make_map8(&mq, q8, d, N, BH)) != FA_OK) return rc;
+    if ((rc = make_map8(&mk, k8, d, N, BH)) != FA_OK) return rc;
+    if ((rc = make_map8(&mv, v8, d, N, BH)) != FA_OK) return rc;
+    if ((rc = make_map(&mo, o, d, N, BH, out_dtype, 128)) != FA_OK) return rc;
+    fa::Fwd8Params p;
+    p.lse = lse;
+    p.sq = sq;
+    p.sk = sk;
+    p.sv = sv;
+    p.N = N;
+    p.nb = (N + 127) / 128;
+    p.nbh = static_cast<int>(BH);
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * kLog2e;
+    using C = fa::Fwd8Cfg;
+    auto kern = out_dtype == FA_BF16 ? fa::fwd8_kernel<true> : fa::fwd8_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(BH * ((p.nb + 1) / 2)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ProfScope prof(6, s);
+    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
                   float scale, int causal, int dtype, void *stream) {

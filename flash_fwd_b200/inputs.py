@@ -94,3 +94,23 @@ def alibi_slopes(H):
     """The geometric head slopes 2^(-8 (h + 1) / H) commonly used with ALiBi (fp32 [H])."""
     return torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32)
 
+
+
+def hadamard_signs(d, seed=0):
+    """float32 [d] of +1/-1 (seeded): the sign flips of the FP8 path's rotation
+    diag(signs) H_d / sqrt(d) (incoherent processing)."""
+    g = torch.Generator().manual_seed(int(seed) + 7919)
+    return (torch.randint(0, 2, (d,), generator=g) * 2 - 1).to(torch.float32)
+
+
+def make_qkv_outliers(B, H, N, d, dtype="bf16", seed=0, channels=4, magnitude=30.0):
+    """Q, K, V i.i.d. N(0, 1) with `channels` outlier channels of Q and K
+    scaled by `magnitude` (the case incoherent processing targets)."""
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    q[..., :channels] *= magnitude
+    k[..., :channels] *= magnitude
+    t = DTYPES[dtype]
+    return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous()

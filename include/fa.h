@@ -217,6 +217,42 @@ FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const voi
                           int B, int H, int N, int d, float scale, int causal, int dtype,
                           void *stream);
 
+/*
+ * FP8 forward with block quantisation and incoherent processing
+ * ("深度解析" section 四: FlashAttention-3's FP8 block quantisation, paired
+ * with incoherent processing to lower the FP8 error).
+ *
+ * fa_fp8_quantize_qkv: q, k, v [B][H][N][d] (DEVICE, dtype FA_F16/FA_BF16,
+ * d in {64, 128, 256}) -> E4M3 codes q8, k8, v8 [B][H][N][d] (DEVICE uint8,
+ * caller-owned) and fp32 scales sq, sk, sv [B][H][ceil(N/128)] (DEVICE):
+ *   - with signs (DEVICE float [d] of +1/-1) Q and K are first multiplied by
+ *     diag(signs) H_d / sqrt(d) (H_d the Sylvester Hadamard matrix), which
+ *     leaves Q K^T unchanged; signs = NULL skips the rotation.  V is never
+ *     rotated.
+ *   - Q and K get one scale per 128-row block, V one per head (stored in every
+ *     block slot of sv): scale = amax / 448, code = E4M3(x * 448 / amax),
+ *     rounded to nearest even and saturating at 448; an all-zero block gets
+ *     scale 1.  The rotation and the quantiser run in fp32 in a fixed operation
+ *     order, so the codes are a pure function of the inputs.
+ * Three launches on `stream`.  Pointers: the tensors 16-byte aligned, the
+ * scales and signs 4-byte aligned.
+ *
+ * fa_fwd_fp8: the forward on those codes (d = 128 only, N = Nq = Nk, causal or
+ * dense, no mask): S = scale * sq * sk * q8 . k8 with fp32 accumulation, the
+ * online softmax in fp32, P rounded to E4M3 for the P V product,
+ * O = sv * sum P8 v8 / sum P8 written as out_dtype (FA_F16/FA_BF16) [B][H][N][d],
+ * lse [B][H][N] fp32 as fa_fwd.  Returns FA_ERR_UNSUPPORTED for d != 128.
+ */
+FA_API int fa_fp8_quantize_qkv(const void *q, const void *k, const void *v,
+                               uint8_t *q8, uint8_t *k8, uint8_t *v8,
+                               float *sq, float *sk, float *sv,
+                               int B, int H, int N, int d, const float *signs, int dtype,
+                               void *stream);
+FA_API int fa_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
+                      const float *sq, const float *sk, const float *sv,
+                      void *o, float *lse, int B, int H, int N, int d,
+                      float scale, int causal, int out_dtype, void *stream);
+
 /* A static, human-readable name for a status code. */
 FA_API const char *fa_status_string(int status);
 
@@ -243,11 +279,11 @@ FA_API int fa_last_timeout_site(int *site);
  * milliseconds and launch counts per kernel kind, clears the record and
  * returns FA_OK.  Kinds: 0 forward, 1 backward pre-pass (D and accumulator
  * reset), 2 backward main kernel, 3 backward dQ conversion, 4 dQ pass of the
- * deterministic backward.  ms and launches
+ * deterministic backward, 5 FP8 quantiser, 6 FP8 forward.  ms and launches
  * are HOST arrays of FA_PROFILE_KINDS entries.  Events are created and
  * destroyed by the library; no device memory is allocated.
  */
-#define FA_PROFILE_KINDS 5
+#define FA_PROFILE_KINDS 7
 FA_API int fa_profile_enable(int on);
 FA_API int fa_profile_read(float *ms, int *launches);
 

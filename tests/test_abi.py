@@ -124,6 +124,27 @@ def test_deterministic_workspace_and_rejects():
     assert det(scale=0.0) == INVALID
 
 
+def test_fp8_entry_points_reject():
+    lib = fa.load_library()
+    F = A   # 16-byte aligned fake device address (no launch happens on these paths)
+
+    def quant(d=128, dtype=1, q=A, sq=F, signs=NULL):
+        return lib.fa_fp8_quantize_qkv(q, A, A, A, A, A, sq, F, F, 1, 1, 128, d, signs, dtype, S)
+
+    def fwd8(d=128, out_dtype=1, o=A, scale=0.1, sq=F):
+        return lib.fa_fwd_fp8(A, A, A, sq, F, F, o, A, 1, 1, 128, d, ctypes.c_float(scale), 0, out_dtype, S)
+    assert quant(q=NULL) == INVALID
+    assert quant(d=96) == UNSUPPORTED
+    assert quant(dtype=7) == INVALID
+    assert quant(q=M) == MISALIGNED
+    assert quant(sq=ctypes.c_void_p(0x10002)) == MISALIGNED
+    assert fwd8(d=64) == UNSUPPORTED          # the FP8 forward is built for d = 128
+    assert fwd8(out_dtype=7) == INVALID
+    assert fwd8(o=M) == MISALIGNED
+    assert fwd8(scale=-1.0) == INVALID
+    assert fwd8(sq=NULL) == INVALID
+
+
 def test_profile_read_rejects_null():
     lib = fa.load_library()
     assert lib.fa_profile_read(None, None) == INVALID
