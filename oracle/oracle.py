@@ -91,7 +91,10 @@ def _mask_arg(mask):
 
 
 def _threads(n):
-    return int(n) if n else (os.cpu_count() or 1)
+    """Threads for one call: n, else ORACLE_THREADS, else every core."""
+    if n:
+        return int(n)
+    return int(os.environ.get("ORACLE_THREADS", "0")) or (os.cpu_count() or 1)
 
 
 def _check_qkv(q, k, v):

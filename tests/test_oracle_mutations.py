@@ -50,22 +50,39 @@ FP8_MUTANTS = {
 
 PIN_FILES = ["test_oracle_pins.py", "test_oracle_modes.py"]
 FP8_PIN_FILES = ["test_oracle_fp8.py"]
+ALL = sorted(MUTANTS) + sorted(FP8_MUTANTS)
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(FP8_MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
-    old, new = MUTANTS[name] if name in MUTANTS else FP8_MUTANTS[name]
-    files = PIN_FILES if name in MUTANTS else FP8_PIN_FILES
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Builds every mutant and runs its pins, all mutants at once (child
+    processes); returns {name: (returncode, tail of the output)}."""
     src = open(SRC).read()
-    assert src.count(old) >= 1, f"mutation anchor not found for {name}"
-    mut = src.replace(old, new)
-    cfile = tmp_path / "oracle_mut.c"
-    cfile.write_text(mut)
-    lib = tmp_path / "liboracle_mut.so"
-    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-I", os.path.join(ROOT, "oracle"),
-                    "-o", str(lib), str(cfile), "-lm", "-lpthread"], check=True)
-    env = dict(os.environ, ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        *[os.path.join(ROOT, "tests", f) for f in files]],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+    procs = {}
+    for name in ALL:
+        old, new = MUTANTS[name] if name in MUTANTS else FP8_MUTANTS[name]
+        files = PIN_FILES if name in MUTANTS else FP8_PIN_FILES
+        assert src.count(old) >= 1, f"mutation anchor not found for {name}"
+        d = tmp_path_factory.mktemp(name)
+        cfile = d / "oracle_mut.c"
+        cfile.write_text(src.replace(old, new))
+        lib = d / "liboracle_mut.so"
+        subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-I", os.path.join(ROOT, "oracle"),
+                        "-o", str(lib), str(cfile), "-lm", "-lpthread"], check=True)
+        # a few oracle threads per child: the children run side by side
+        env = dict(os.environ, ORACLE_LIB=str(lib), ORACLE_THREADS="2")
+        procs[name] = subprocess.Popen([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                                        *[os.path.join(ROOT, "tests", f) for f in files]],
+                                       cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                       text=True)
+    out = {}
+    for name, pr in procs.items():
+        text, _ = pr.communicate(timeout=900)
+        out[name] = (pr.returncode, text[-2000:])
+    return out
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_pins_catch_mutant(name, mutant_runs):
+    rc, tail = mutant_runs[name]
+    assert rc != 0, f"mutant {name} survived the pins:\n{tail}"
