@@ -324,7 +324,9 @@ def run_reference(args, w, name):
         secs += oracle_head_pass(host, w, (args.warmup + i) % (w["B"] * w["H"]))
     val = args.steps * per_head_flops(w, kept) / secs / 1e12
     cores = os.cpu_count()
-    sample = f"one (batch, head) of the workload per step: forward on all {w['N']} rows, dQ on all rows, dK/dV on all keys"
+    what = ("E4M3 quantisation and the FP8 forward on all rows" if w.get("fp8") else
+            "forward on all rows, dQ on all rows, dK/dV on all keys" if w["bwd"] else "forward on all rows")
+    sample = f"one (batch, head) of the workload per step ({w['N']} rows): {what}"
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
@@ -477,9 +479,10 @@ def run_ours(args, w, name):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads, secs, val = cpu_sample(host, w, kept, args.cpu_seconds)
+        what = ("E4M3 quantisation of Q, K, V and the FP8 forward on all rows" if w.get("fp8") else
+                "forward on all rows, dQ on all rows, dK/dV on all keys" if w["bwd"] else "forward on all rows")
         cpu = {"value": val, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
-               "sample": f"{heads} of {w['B'] * w['H']} (batch, head) pairs, each: forward on all rows, "
-                         f"dQ on all rows, dK/dV on all keys; {secs:.1f} s"}
+               "sample": f"{heads} of {w['B'] * w['H']} (batch, head) pairs, each: {what}; {secs:.1f} s"}
 
     in_bytes = sum(x.numel() * x.element_size() for x in (t["q"], t["k"], t["v"]) + ((t["do"],) if w["bwd"] else ()))
     line = {
