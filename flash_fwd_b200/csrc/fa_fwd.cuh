@@ -21,7 +21,9 @@
 //                       row.  It reads S_t from TMEM, masks, updates m and l,
 //                       rescales O_t in TMEM when m grew by more than 2^8
 //                       (exactness is kept because O and l share the stale m),
-//                       writes P_t (16-bit) back over S_t and signals the MMA warp.
+//                       writes P_t (16-bit) back over S_t and signals the MMA
+//                       warp once per half (keys 0..63, 64..127): O_t += P_t V
+//                       starts on the first half while the second is computed.
 //   warp 4*NQ           TMA producer: Q tiles once, then K_j per stage (and
 //                       V_j when NQ = 1).
 //   warp 4*NQ+2         (NQ = 2) TMA producer of the V_j tiles.
@@ -119,7 +121,8 @@ struct FwdCfg {
     static constexpr int kBarSFull = kBarVEmpty + NSV;
     static constexpr int kBarPFull = kBarSFull + NQ;
     static constexpr int kBarOFull = kBarPFull + NQ;
-    static constexpr int kBarMmaDone = kBarOFull + NQ;
+    static constexpr int kBarPFull2 = kBarOFull + NQ;   // P_t keys 64..127 in TMEM (kBarPFull: keys 0..63)
+    static constexpr int kBarMmaDone = kBarPFull2 + NQ;
     static constexpr int kNumBars = kBarMmaDone + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + slack for 1 KB alignment
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         for (int t = 0; t < NQ; ++t) {
             mbar_init(bar(C::kBarSFull + t), 1);
             mbar_init(bar(C::kBarPFull + t), 128);
+            mbar_init(bar(C::kBarPFull2 + t), 128);
             mbar_init(bar(C::kBarOFull + t), 1);
         }
         mbar_init(bar(C::kBarMmaDone), 1);
@@ -288,11 +292,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                            k > 0 ? 1u : 0u, leader);
                 }
             };
-            auto issue_pv = [&](int t, int s, bool acc) {
+            auto issue_pv = [&](int t, int s, bool acc, int k0, int k1) {
                 const uint32_t d_tmem = tmem + C::kOCol + D * t;
                 const uint32_t a_tmem = tmem + 128u * t;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
+                for (int k = k0; k < k1; ++k)
                     mma_ts(d_tmem, a_tmem + 8u * k, dV.at(s * C::kTileBytes + k * 2048), kIdescO,
                            (acc || k > 0) ? 1u : 0u, leader);
             };
@@ -337,7 +341,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                         ok = wait_bar(bar(C::kBarPFull + t), cnt[t] & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_pv(t, s, cnt[t] > 0);
+                        issue_pv(t, s, cnt[t] > 0, 0, 4);
+                        __syncwarp();
+                        ok = wait_bar(bar(C::kBarPFull2 + t), cnt[t] & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(t, s, cnt[t] > 0, 4, 8);
                         __syncwarp();
                         ++cnt[t];
                     }
@@ -486,6 +495,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     }
                 }
                 tmem_st16(tS + 16 * q, pk);
+                if (q == 1) {
+                    // the first 64 keys of P_t are in TMEM: the MMA warp can start
+                    // O_t += P_t V on them while the second half is computed
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarPFull + t));
+                }
             }
             const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
             const float sum = s01.x + s01.y;
@@ -499,7 +515,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             m = m_new;
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull + t));
+            mbar_arrive(bar(C::kBarPFull2 + t));
             ++cnt;
         }
         if (ok && cnt > 0) ok = wait_bar(bar(C::kBarOFull + t), 0, abort_flag);
