@@ -126,11 +126,13 @@ __global__ void __launch_bounds__(QuantCfg<D>::kThreads)
                     }
 #pragma unroll
             for (int h = E; h < D; h <<= 1) {              // across lanes: lane ^ (h / E)
-                const bool lower = (lane & (h / E)) == 0;
+                // lower lane: x + y; upper lane: y - x, as one exactly rounded
+                // fma(+-1, x, y) (the same result as the add or the subtraction)
+                const float sgn = (lane & (h / E)) == 0 ? 1.0f : -1.0f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
                     const float y = __shfl_xor_sync(0xffffffffu, x[r][e], h / E);
-                    x[r][e] = lower ? x[r][e] + y : y - x[r][e];
+                    x[r][e] = fmaf(sgn, x[r][e], y);
                 }
             }
 #pragma unroll
