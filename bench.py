@@ -118,6 +118,19 @@ def describe(name, w):
     return s
 
 
+def device_info(index):
+    """GPU name, driver and CUDA runtime of this rank's device."""
+    import torch
+    info = {"name": torch.cuda.get_device_name(index), "cuda_runtime": torch.version.cuda, "driver": None}
+    try:
+        r = subprocess.run(["nvidia-smi", "-i", str(index), "--query-gpu=driver_version", "--format=csv,noheader"],
+                           capture_output=True, text=True, timeout=20)
+        info["driver"] = r.stdout.strip() or None
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return info
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "flash_fwd_b200", "csrc", "*.cu*"))):
@@ -449,6 +462,38 @@ def run_ours(args, w, name):
         split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12
         split["bwd_frac_of_peak"] = split["bwd_tflops"] / peak
 
+    # ---------------- the same steps replayed from a CUDA graph (launch overhead removed)
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step(w, t, side)                      # warm the capture stream once
+        stream.wait_stream(side)
+        torch.cuda.synchronize(device)
+        with torch.cuda.graph(g):
+            cap = torch.cuda.current_stream(device)
+            for _ in range(args.steps):
+                step(w, t, cap)
+        torch.cuda.synchronize(device)
+        g.replay()
+        torch.cuda.synchronize(device)
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(device)
+        gms = g0.elapsed_time(g1)
+        graph = {"ms_per_step": gms / args.steps, "value": flops * args.steps / (gms / 1e3) / 1e12, "unit": UNIT,
+                 "steps_per_replay": args.steps}
+        del g
+        if fa.fa_last_device_status() != 0:
+            raise RuntimeError("device status after the graph replay is not ok")
+    except RuntimeError as e:   # capture refused or failed: reported, not fatal
+        graph = {"error": str(e)[:200]}
+
     # ---------------- end to end through host buffers
     e2e = None
     if args.e2e_steps > 0:
@@ -501,6 +546,8 @@ def run_ours(args, w, name):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
+        "graph": graph,
+        "device": device_info(local),
         "gpu_launches": sum(v[1] for v in prof.values()),
     }
     if rank == 0:
