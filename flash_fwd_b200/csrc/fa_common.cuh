@@ -438,7 +438,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // degree-3 minimax polynomial in relative error produced by
 // gen_exp2_poly.py (max relative error 7.5e-5); 2^j enters the exponent
 // field by an integer add.  x is clamped to [-125, +inf): below that the
-// true value is < 2^-124 and the result stays a tiny positive normal.
+// true value is < 2^-124 and the result stays a tiny positive normal -- also
+// for x = -inf (a masked score), which the caller must account for.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     constexpr float kRound = 12582912.0f;                 // 1.5 * 2^23
     constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f;

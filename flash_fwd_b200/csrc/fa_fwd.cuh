@@ -36,9 +36,8 @@
 // Scale handling: exp is evaluated as 2^(s * scale * log2 e - m), with the
 // running max m kept in that base-2 domain; LSE converts back to natural log.
 // exp2 runs on the special-function unit (16 results per clock per SM); a
-// degree-3 polynomial on the FMA pipe (128 per clock) can take a share of the
-// pairs (kPolyPairs), which measured slower here because the softmax warps
-// are issue-bound.
+// degree-3 polynomial on the FMA pipe (128 per clock) can take a share of
+// the pairs (kPolyPairs); it is off (see the softmax loop for the measurements).
 #pragma once
 
 #include "fa_common.cuh"
@@ -462,10 +461,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     tmem_st32(tO + 32 * q, o);
                 }
             }
-            // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA pipe
-            // (polynomial) instead of the special-function unit; measured on
-            // B200 the softmax is issue-bound rather than MUFU-bound here, and
-            // moving any pairs made it slower, so all of them use MUFU.
+            // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA
+            // pipe (polynomial) instead of the special-function unit.  Measured
+            // on B200: at d = 128 and 256 moving any pairs made the softmax
+            // slower (issue-bound); at d = 64 two of eight were 4.7 % faster
+            // but failed the parity of a causal cross-attention case (Nq = 300,
+            // Nk = 100) not yet explained, so every pair uses the special-
+            // function unit.
             constexpr int kPolyPairs = 0;
             float2 acc[4], acc_r[4];
 #pragma unroll
@@ -528,7 +530,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         if (epi) {
             const bool valid = row < p.Nq;
             const float l_o = BF16 ? l_r : l;
-            const float inv_l = (cnt > 0 && l_o > 0.f) ? 1.0f / l_o : 0.0f;
+            // m = -inf: the row saw no key.  (The polynomial exp2 gives 2^-125,
+            // not 0, for masked scores, so l alone would not tell.)
+            const float inv_l = (cnt > 0 && l_o > 0.f && m != -INFINITY) ? 1.0f / l_o : 0.0f;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
