@@ -568,13 +568,15 @@ __global__ void __launch_bounds__(512, 1)
                 const float mul = is_dv ? 1.0f : p.scale;
                 uint8_t *stage = smem + (is_dv ? C::kVOff : C::kKOff);
                 const uint32_t col0 = is_dv ? C::kColDV : C::kColDK;
+                // a key block that no query tile sees never waited for its K/V
+                // loads: they must land before the staging areas are written
+                if (done && cnt == 0) drain_bar(bar(C::kBarKV), 0);
                 if (done) {
         #pragma unroll 1
                     for (int ch = 0; ch < D / 32; ++ch) {
                         uint32_t v[32];
                         if (cnt > 0) {
-                            tmem_ld32(tmem + lane_off + col0 + 32 * ch, v);
-                            tmem_ld_wait();
+                            tmem_ld32_wait(tmem + lane_off + col0 + 32 * ch, v);
                         } else {
     #pragma unroll
                             for (int k = 0; k < 32; ++k) v[k] = 0u;   // no query sees this key block
@@ -616,6 +618,9 @@ __global__ void __launch_bounds__(512, 1)
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t v[BM];
+                // 128 registers: four loads and one wait (a single load-and-wait
+                // statement does not fit this kernel's register budget); v is
+                // only read after the wait
 #pragma unroll
                 for (int ch = 0; ch < BM / 32; ++ch)
                     tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));

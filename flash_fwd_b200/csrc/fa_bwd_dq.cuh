@@ -489,14 +489,16 @@ __global__ void __launch_bounds__(352, 1)
         bool done = ok;
         if (done && cnt > 0) done = wait_bar(bar(C::kBarMmaDone), 0, abort_flag);
         tc_fence_after();
+        // a tile that sees no key block never waited for its Q/dO loads: they
+        // must land before the staging area (the Q buffer) is written
+        if (done && cnt == 0) drain_bar(bar(C::kBarQ), 0);
         if (done) {
             // this thread: row `row`, d columns [kh D / 2, (kh + 1) D / 2)
 #pragma unroll 1
             for (int ch = 0; ch < D / 64; ++ch) {
                 uint32_t v[32];
                 if (cnt > 0) {
-                    tmem_ld32(tmem + lane_off + C::kColDQ + kh * (D / 2) + 32 * ch, v);
-                    tmem_ld_wait();
+                    tmem_ld32_wait(tmem + lane_off + C::kColDQ + kh * (D / 2) + 32 * ch, v);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] = 0u;   // a tile that sees no key: dQ = 0

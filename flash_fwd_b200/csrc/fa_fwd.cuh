@@ -406,10 +406,16 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             tc_fence_after();
             uint32_t r[128];
 #pragma unroll
+#pragma unroll
             for (int q = 0; q < 4; ++q)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
             tmem_ld_wait();
-            float *sv = reinterpret_cast<float *>(r);
+            // the scores as floats: a copy, not a float* view of r (reading
+            // the asm-written integers through another type is undefined and
+            // let stale register values into the row max)
+            float sv[128];
+#pragma unroll
+            for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
             // this row's visible keys within the tile: [lo, hi]
             int lo, hi, rk = 0;
             if constexpr (GENERAL) {
@@ -454,8 +460,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
 #pragma unroll 1
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t o[32];
-                    tmem_ld32(tO + 32 * q, o);
-                    tmem_ld_wait();
+                    tmem_ld32_wait(tO + 32 * q, o);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
                     tmem_st32(tO + 32 * q, o);
@@ -527,6 +532,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         // TMA stores: one thread per row would touch 32 lines per store
         const bool epi = rb < p.nqb && ok;
         uint8_t *stage = smem + C::kQOff + t * C::kTileBytes;
+        // a tile that saw no key block never waited for its Q load: it must
+        // land before the staging area is written
+        if (epi && cnt == 0) drain_bar(bar(C::kBarQ), 0);
         if (epi) {
             const bool valid = row < p.Nq;
             const float l_o = BF16 ? l_r : l;
@@ -537,8 +545,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
                 if (cnt > 0) {
-                    tmem_ld32(tO + 32 * q, o);
-                    tmem_ld_wait();
+                    tmem_ld32_wait(tO + 32 * q, o);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = 0u;

@@ -439,10 +439,16 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
             uint32_t r[128];
 #pragma unroll
+#pragma unroll
             for (int q = 0; q < 4; ++q)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
             tmem_ld_wait();
-            float *sv = reinterpret_cast<float *>(r);
+            // the scores as floats: a copy, not a float* view of r (reading
+            // the asm-written integers through another type is undefined and
+            // let stale register values into the row max)
+            float sv[128];
+#pragma unroll
+            for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
             int hi = 127;
             if (p.causal && j == rb) hi = row_local;                          // diagonal tile
             if (j == p.nb - 1 && (p.N & 127)) hi = min(hi, (p.N & 127) - 1);  // key tail
@@ -469,8 +475,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 1
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t o[32];
-                    tmem_ld32(tO + 32 * q, o);
-                    tmem_ld_wait();
+                    tmem_ld32_wait(tO + 32 * q, o);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
                     tmem_st32(tO + 32 * q, o);
@@ -517,8 +522,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
                 if (cnt > 0) {
-                    tmem_ld32(tO + 32 * q, o);
-                    tmem_ld_wait();
+                    tmem_ld32_wait(tO + 32 * q, o);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = 0u;
