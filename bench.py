@@ -207,12 +207,11 @@ class ClockSampler:
 
 
 def power_capped(clocks):
-    """True when the timed region ran under the power cap (reason seen, or SM
-    clocks sampled well below their maximum)."""
+    """True when the power cap actually slowed the timed region: SM clocks
+    sampled below 95 % of their maximum.  The sw_power_cap flag alone, with
+    the clock still at its maximum, keeps the burst peak."""
     if not clocks or clocks.get("sm_mhz") is None:
         return False
-    if "sw_power_cap" in clocks.get("reasons", []):
-        return True
     mx = clocks.get("sm_max_mhz") or 0
     return bool(mx) and clocks.get("sm_min_mhz", mx) < 0.95 * mx
 
