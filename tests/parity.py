@@ -79,12 +79,14 @@ def check_fwd(o_gpu, lse_gpu, q, k, v, causal, scale, dtype, mask=None, rows_per
     return worst_o, worst_l
 
 
-def check_bwd(grads_gpu, q, k, v, do, causal, scale, mask=None, dq_rows=None, kv_cols=None, heads=None, seed=0):
+def check_bwd(grads_gpu, q, k, v, do, causal, scale, mask=None, dq_rows=None, kv_cols=None, heads=None, seed=0,
+              kv_blocks=None):
     """Compares dQ, dK, dV with the oracle.
 
     Full check when dq_rows is None; otherwise dQ on `dq_rows` sampled rows per
-    head and dK/dV on `kv_cols` sampled keys per head, for the heads listed in
-    `heads` (all when None).  Bar: max |err| <= 5e-2 * max |oracle value|.
+    head and dK/dV on `kv_cols` sampled keys per head -- or, with kv_blocks, on
+    every key of `kv_blocks` sampled 128-key block columns per head -- for the
+    heads listed in `heads` (all when None).  Bar: max |err| <= 5e-2 * max |oracle value|.
     """
     B, H, N, d = q.shape
     Q, K, V, DO = bh(q), bh(k), bh(v), bh(do)
@@ -103,7 +105,11 @@ def check_bwd(grads_gpu, q, k, v, do, causal, scale, mask=None, dq_rows=None, kv
         worst = {"dq": [0.0, 0.0], "dk": [0.0, 0.0], "dv": [0.0, 0.0]}
         for hh in hs:
             rows = inputs.sample_rows(N, dq_rows, seed, hh).numpy()
-            cols = inputs.sample_rows(N, kv_cols, seed + 7, hh).numpy()
+            if kv_blocks is None:
+                cols = inputs.sample_rows(N, kv_cols, seed + 7, hh).numpy()
+            else:
+                blocks = inputs.sample_key_blocks((N + 127) // 128, kv_blocks, seed, hh).numpy()
+                cols = np.concatenate([np.arange(b * 128, min(b * 128 + 128, N)) for b in blocks]).astype(np.int32)
             sl = slice(hh, hh + 1)
             rdq = oracle.bwd_dq_rows(Q[sl], K[sl], V[sl], DO[sl], scale, rows, fl, mk)[0]
             rdk, rdv = oracle.bwd_dkdv_cols(Q[sl], K[sl], V[sl], DO[sl], scale, cols, fl, mk)

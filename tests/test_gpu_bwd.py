@@ -62,7 +62,19 @@ def test_bwd_sparse64k_config_sampled():
     mask = inputs.make_block_mask(c["N"], 128, c["density"], seed=0)
     scale = inputs.default_scale(c["d"])
     _, _, grads = _run(q, k, v, do, False, scale, mask)
-    check_bwd(grads, q, k, v, do, False, scale, mask=mask, dq_rows=128, kv_cols=64)
+    # 256 query rows per head for dQ; dK/dV on every key of 2 key-block columns per head
+    check_bwd(grads, q, k, v, do, False, scale, mask=mask, dq_rows=256, kv_blocks=2)
+
+
+def test_sparse_2048_full():
+    # the same mask generator at N = 2048: forward and backward checked on every element
+    N, d = 2048, 64
+    q, k, v, do = inputs.make_qkv(1, 4, N, d, "bf16", seed=0)
+    mask = inputs.make_block_mask(N, 128, 0.2, seed=0)
+    scale = inputs.default_scale(d)
+    o, lse, grads = _run(q, k, v, do, False, scale, mask)
+    check_fwd(o, lse, q, k, v, False, scale, "bf16", mask=mask)
+    check_bwd(grads, q, k, v, do, False, scale, mask=mask)
 
 
 @pytest.mark.parametrize("causal", [False, True])
