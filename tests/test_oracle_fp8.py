@@ -191,3 +191,20 @@ def test_incoherent_processing_lowers_the_error():
         o, _ = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv[:, 0], scale)
         errs[name] = np.sqrt(np.mean((o - ref) ** 2))
     assert errs["incoherent"] * 1.5 < errs["plain"], errs
+
+
+def test_quantizer_matches_numpy_and_torch_float8():
+    # the quantiser without rotation, written with numpy fp32 arithmetic and
+    # PyTorch's float8_e4m3fn cast: the same scales and codes
+    g = np.random.default_rng(6)
+    BH, N, d = 2, 300, 128
+    x = (g.normal(0, 1, (BH, N, d)) * g.uniform(0.001, 50, (BH, N, 1))).astype(np.float32)
+    codes, scales = oracle.fp8_quantize(x, 128)
+    for h in range(BH):
+        for b in range(3):
+            blk = x[h, b * 128:(b + 1) * 128]
+            amax = np.float32(np.abs(blk).max())
+            assert scales[h, b] == np.float32(amax / np.float32(448.0))
+            y = (blk * (np.float32(448.0) / amax)).astype(np.float32)
+            ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(codes[h, b * 128:(b + 1) * 128], ref)
