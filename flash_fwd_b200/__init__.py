@@ -17,6 +17,7 @@ __all__ = [
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
     "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes", "fa_bwd_deterministic",
     "fa_bwd_deterministic_workspace_bytes", "fa_fp8_quantize_qkv", "fa_fwd_fp8", "attention_fwd_fp8",
+    "fa_bwd_noalloc",
 ]
 
 FA_BLOCK = 128
@@ -62,6 +63,7 @@ def load_library():
     lib.fa_bwd_deterministic.argtypes = list(lib.fa_bwd_ex.argtypes)
     lib.fa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, i, vp]
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, f, i, i, vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -70,7 +72,7 @@ def load_library():
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
-               lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8,
+               lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8, lib.fa_bwd_noalloc,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -214,6 +216,15 @@ def fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=
                                   B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)), wl, wr, _ptr(alibi_slopes),
                                   _ptr(block_mask), _dtype(q), _stream(stream))
     _check(rc, "fa_bwd_ex")
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, causal=False, scale=None, stream=None):
+    """fa_bwd without a workspace: the library's own device scratch serves (see include/fa.h)."""
+    B, H, N, d = _shape(q)
+    rc = load_library().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                       _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q),
+                                       _stream(stream))
+    _check(rc, "fa_bwd_noalloc")
 
 
 def fa_bwd_deterministic_workspace_bytes(B, H, Nq, Nk, d):

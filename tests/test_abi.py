@@ -33,6 +33,26 @@ def test_library_loads_and_exports_every_declared_function():
         assert hasattr(lib, n), f"{n} declared in fa.h but not exported"
 
 
+def declared_arity():
+    """{function: number of parameters} from the declarations in fa.h."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    lib = fa.load_library()
+    arity = declared_arity()
+    assert set(arity) == set(declared_functions())
+    for name, n in arity.items():
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, f"{name}: the binding sets no argtypes"
+        assert len(argtypes) == n, f"{name}: header has {n} parameters, binding {len(argtypes)}"
+
+
 def test_status_strings():
     for code in range(0, 8):
         assert isinstance(fa.fa_status_string(code), str) and fa.fa_status_string(code)
