@@ -67,6 +67,8 @@ WORKLOADS = {
 
 def general(w):
     return "Nk" in w or "window" in w or w.get("alibi", False)
+
+
 L2_BYTES = 126 * 1024 * 1024
 
 
