@@ -123,6 +123,59 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _on_device(t):
+    """Is t in device memory of the current device (where the library launches)?"""
+    return t.is_cuda and t.device.index == torch.cuda.current_device()
+
+
+_HALF = (torch.float16, torch.bfloat16)
+_F32 = (torch.float32,)
+_U8 = (torch.uint8,)
+
+
+def _need(name, t, dtypes=None, shape=None, numel=None):
+    """Checks one tensor argument before its address goes to the library, which
+    cannot check a pointer: a contiguous tensor in the current device's memory,
+    of an accepted dtype and of the given shape (or element count).  Raises
+    TypeError / ValueError; nothing is launched."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if not _on_device(t):
+        raise ValueError(f"{name}: must be a CUDA tensor on the current device (got {t.device})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not accepted ({', '.join(str(x) for x in dtypes)})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+
+
+def _need_attention(q, k, v, o, lse, square, dout=None, dq=None, dk=None, dv=None, workspace=None,
+                    block_mask=None, alibi_slopes=None):
+    """Checks the tensors of one attention call; returns (B, H, Nq, Nk, d)."""
+    _need("q", q, _HALF)
+    B, H, Nq, d = _shape(q)
+    _need("k", k, (q.dtype,))
+    if k.dim() != 4 or tuple(k.shape[:2]) != (B, H) or int(k.shape[3]) != d or (square and k.shape[2] != Nq):
+        raise ValueError(f"k: shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    Nk = int(k.shape[2])
+    _need("v", v, (q.dtype,), shape=k.shape)
+    _need("o", o, (q.dtype,), shape=q.shape)
+    _need("lse", lse, _F32, numel=B * H * Nq)
+    for name, t, like in (("dout", dout, q), ("dq", dq, q), ("dk", dk, k), ("dv", dv, k)):
+        if t is not None:
+            _need(name, t, (q.dtype,), shape=like.shape)
+    if workspace is not None:
+        _need("workspace", workspace)          # its size is the library's check
+    if block_mask is not None:
+        _need("block_mask", block_mask, _U8, numel=((Nq + 127) // 128) * ((Nk + 127) // 128))
+    if alibi_slopes is not None:
+        _need("alibi_slopes", alibi_slopes, _F32, numel=H)
+    return B, H, Nq, Nk, d
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -152,14 +205,14 @@ def _check(rc, what):
 
 def fa_fwd(q, k, v, o, lse, causal=False, scale=None, stream=None):
     """O and LSE of exact attention; all tensors [B, H, N, d] (lse [B, H, N] fp32)."""
-    B, H, N, d = _shape(q)
+    B, H, N, _, d = _need_attention(q, k, v, o, lse, square=True)
     rc = load_library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                                _scale(scale, d), int(bool(causal)), _dtype(q), _stream(stream))
     _check(rc, "fa_fwd")
 
 
 def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, causal=False, scale=None, stream=None):
-    B, H, N, d = _shape(q)
+    B, H, N, _, d = _need_attention(q, k, v, o, lse, square=True, block_mask=block_mask)
     rc = load_library().fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask),
                                            B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q),
                                            _stream(stream))
@@ -167,7 +220,7 @@ def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, causal=False, scale=None, st
 
 
 def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, stream=None):
-    B, H, N, d = _shape(q)
+    B, H, N, _, d = _need_attention(q, k, v, o, lse, True, dout, dq, dk, dv, workspace)
     rc = load_library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q), _stream(stream))
@@ -176,7 +229,7 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=Non
 
 def fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, block_mask, causal=False, scale=None,
                        stream=None):
-    B, H, N, d = _shape(q)
+    B, H, N, _, d = _need_attention(q, k, v, o, lse, True, dout, dq, dk, dv, workspace, block_mask)
     rc = load_library().fa_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                                            _ptr(dk), _ptr(dv), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), _ptr(block_mask),
@@ -193,8 +246,7 @@ def fa_fwd_ex(q, k, v, o, lse, causal=False, scale=None, window=None, alibi_slop
               stream=None):
     """General forward: q, o [B, H, Nq, d]; k, v [B, H, Nk, d]; lse [B, H, Nq] fp32.
     window=(left, right) (a negative side is unbounded), alibi_slopes: fp32 [H] on the device."""
-    B, H, Nq, d = _shape(q)
-    Nk = int(k.shape[2])
+    B, H, Nq, Nk, d = _need_attention(q, k, v, o, lse, False, block_mask=block_mask, alibi_slopes=alibi_slopes)
     wl, wr = _window(window)
     rc = load_library().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
                                   _scale(scale, d), int(bool(causal)), wl, wr, _ptr(alibi_slopes), _ptr(block_mask),
@@ -208,8 +260,8 @@ def fa_bwd_ex_workspace_bytes(B, H, Nq, Nk, d):
 
 def fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, window=None,
               alibi_slopes=None, block_mask=None, stream=None):
-    B, H, Nq, d = _shape(q)
-    Nk = int(k.shape[2])
+    B, H, Nq, Nk, d = _need_attention(q, k, v, o, lse, False, dout, dq, dk, dv, workspace, block_mask,
+                                      alibi_slopes)
     wl, wr = _window(window)
     rc = load_library().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                   _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -220,7 +272,7 @@ def fa_bwd_ex(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=
 
 def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, causal=False, scale=None, stream=None):
     """fa_bwd without a workspace: the library's own device scratch serves (see include/fa.h)."""
-    B, H, N, d = _shape(q)
+    B, H, N, _, d = _need_attention(q, k, v, o, lse, True, dout, dq, dk, dv)
     rc = load_library().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                        _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(q),
                                        _stream(stream))
@@ -234,8 +286,8 @@ def fa_bwd_deterministic_workspace_bytes(B, H, Nq, Nk, d):
 def fa_bwd_deterministic(q, k, v, o, dout, lse, dq, dk, dv, workspace, causal=False, scale=None, window=None,
                          alibi_slopes=None, block_mask=None, stream=None):
     """fa_bwd_ex with bitwise reproducible outputs (dQ by a second sweep, no atomics)."""
-    B, H, Nq, d = _shape(q)
-    Nk = int(k.shape[2])
+    B, H, Nq, Nk, d = _need_attention(q, k, v, o, lse, False, dout, dq, dk, dv, workspace, block_mask,
+                                      alibi_slopes)
     wl, wr = _window(window)
     rc = load_library().fa_bwd_deterministic(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
@@ -291,7 +343,12 @@ def fa_fp8_quantize_qkv(q, k, v, signs=None, stream=None):
     """E4M3 codes and scales of q, k, v [B, H, N, d] (16-bit, on the device):
     returns (q8, k8, v8 uint8 [B, H, N, d], sq, sk, sv fp32 [B, H, ceil(N / 128)]).
     signs (fp32 [d] of +-1 on the device) rotates Q and K by diag(signs) H_d / sqrt(d)."""
+    _need("q", q, _HALF)
     B, H, N, d = _shape(q)
+    _need("k", k, (q.dtype,), shape=q.shape)
+    _need("v", v, (q.dtype,), shape=q.shape)
+    if signs is not None:
+        _need("signs", signs, _F32, numel=d)
     nb = (N + 127) // 128
     q8, k8, v8 = (torch.empty((B, H, N, d), dtype=torch.uint8, device=q.device) for _ in range(3))
     sq, sk, sv = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
@@ -304,7 +361,15 @@ def fa_fp8_quantize_qkv(q, k, v, signs=None, stream=None):
 def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal=False, scale=None, stream=None):
     """FP8 forward on the codes and scales of fa_fp8_quantize_qkv; o [B, H, N, d]
     (float16 or bfloat16) and lse [B, H, N] fp32 are written."""
+    _need("q8", q8, _U8)
     B, H, N, d = _shape(q8)
+    nb = (N + 127) // 128
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _need(name, t, _U8, shape=q8.shape)
+    for name, t in (("sq", sq), ("sk", sk), ("sv", sv)):
+        _need(name, t, _F32, numel=B * H * nb)
+    _need("o", o, _HALF, shape=q8.shape)
+    _need("lse", lse, _F32, numel=B * H * N)
     rc = load_library().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
                                    B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(o), _stream(stream))
     _check(rc, "fa_fwd_fp8")
