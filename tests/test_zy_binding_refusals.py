@@ -1,7 +1,8 @@
-"""(Collected next to last, before the no-alloc tests.)  The binding refuses, with real device tensors, what the C ABI could not
+"""The binding refuses, with real device tensors, what the C ABI could not
 check: a host tensor among device ones, a strided view, a short output, a
 mismatched dtype.  Nothing is launched, so the device status stays 0, and a
-well-formed call right after still runs.
+well-formed call right after still runs.  (Collected next to last, before
+the no-alloc tests.)
 """
 import pytest
 import torch
