@@ -278,7 +278,8 @@ def step(w, t, stream):
 # --------------------------------------------------------------------------
 def oracle_head_pass(host, w, head):
     """One (batch, head) of the workload through the fp64 oracle: forward on
-    every row, dQ on every row, dK/dV on every key.  Returns seconds."""
+    every row, dQ on every row, dK/dV on every key.  Returns the seconds of
+    the forward and of the backward."""
     import numpy as np
 
     import oracle
@@ -300,14 +301,15 @@ def oracle_head_pass(host, w, head):
         k8, sk = oracle.fp8_quantize(K.astype(np.float32), 128, signs)
         v8, sv = oracle.fp8_quantize(V.astype(np.float32), N)
         oracle.fwd_fp8(q8, k8, v8, sq, sk, sv[:, 0], 1.0 / d ** 0.5, causal=w["causal"])
-        return time.perf_counter() - t0
+        return time.perf_counter() - t0, 0.0
     t0 = time.perf_counter()
     oracle.fwd_rows(Q, K, V, 1.0 / d ** 0.5, flags, mask, 128, rows, **modes)
+    t1 = time.perf_counter()
     if w["bwd"]:
         DO = sl(host["do"], N)
         oracle.bwd_dq_rows(Q, K, V, DO, 1.0 / d ** 0.5, rows, flags, mask, 128, **modes)
         oracle.bwd_dkdv_cols(Q, K, V, DO, 1.0 / d ** 0.5, cols, flags, mask, 128, **modes)
-    return time.perf_counter() - t0
+    return t1 - t0, time.perf_counter() - t1
 
 
 def per_head_flops(w, kept_blocks):
@@ -316,12 +318,24 @@ def per_head_flops(w, kept_blocks):
 
 
 def cpu_sample(host, w, kept_blocks, budget_s, max_heads=None):
+    """Whole (batch, head) passes of the oracle until the budget is spent (at
+    least one).  Returns (heads, seconds, TFLOP/s, forward s, backward s)."""
     heads = w["B"] * w["H"] if max_heads is None else min(max_heads, w["B"] * w["H"])
-    done, secs = 0, 0.0
-    while done < heads and (secs < budget_s or done == 0):
-        secs += oracle_head_pass(host, w, done)
+    done, tf, tb = 0, 0.0, 0.0
+    while done < heads and (tf + tb < budget_s or done == 0):
+        f, b = oracle_head_pass(host, w, done)
+        tf, tb = tf + f, tb + b
         done += 1
-    return done, secs, done * per_head_flops(w, kept_blocks) / secs / 1e12
+    secs = tf + tb
+    return done, secs, done * per_head_flops(w, kept_blocks) / secs / 1e12, tf, tb
+
+
+def oracle_seconds(w, heads, tf, tb):
+    """The oracle's forward and backward wall-clock seconds per (batch, head),
+    and the whole workload's, extrapolated from the sampled heads."""
+    per_f, per_b = tf / heads, tb / heads
+    return {"fwd_s_per_head": per_f, "bwd_s_per_head": per_b if w["bwd"] else None,
+            "extrapolated_full_workload_s": (per_f + per_b) * w["B"] * w["H"]}
 
 
 def run_reference(args, w, name):
@@ -333,9 +347,11 @@ def run_reference(args, w, name):
     kept = int(host["mask"].sum()) if w["sparse"] else None
     for i in range(args.warmup):
         oracle_head_pass(host, w, i % (w["B"] * w["H"]))
-    secs = 0.0
+    tf = tb = 0.0
     for i in range(args.steps):
-        secs += oracle_head_pass(host, w, (args.warmup + i) % (w["B"] * w["H"]))
+        f, b = oracle_head_pass(host, w, (args.warmup + i) % (w["B"] * w["H"]))
+        tf, tb = tf + f, tb + b
+    secs = tf + tb
     val = args.steps * per_head_flops(w, kept) / secs / 1e12
     cores = os.cpu_count()
     what = ("E4M3 quantisation and the FP8 forward on all rows" if w.get("fp8") else
@@ -346,7 +362,8 @@ def run_reference(args, w, name):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": describe(name, w), "per_step": "one (batch, head)"},
-        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         **oracle_seconds(w, args.steps, tf, tb)},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -541,11 +558,12 @@ def run_ours(args, w, name):
     # ---------------- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        heads, secs, val = cpu_sample(host, w, kept, args.cpu_seconds)
+        heads, secs, val, tf, tb = cpu_sample(host, w, kept, args.cpu_seconds)
         what = ("E4M3 quantisation of Q, K, V and the FP8 forward on all rows" if w.get("fp8") else
                 "forward on all rows, dQ on all rows, dK/dV on all keys" if w["bwd"] else "forward on all rows")
         cpu = {"value": val, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
-               "sample": f"{heads} of {w['B'] * w['H']} (batch, head) pairs, each: {what}; {secs:.1f} s"}
+               "sample": f"{heads} of {w['B'] * w['H']} (batch, head) pairs, each: {what}; {secs:.1f} s",
+               **oracle_seconds(w, heads, tf, tb)}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -31,6 +31,9 @@ def test_reference_arm_line(workload):
     assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    # the oracle's forward and backward seconds per (batch, head), and the whole workload extrapolated
+    assert cb["fwd_s_per_head"] > 0 and cb["extrapolated_full_workload_s"] > cb["fwd_s_per_head"]
+    assert (cb["bwd_s_per_head"] is None) == (not bench.WORKLOADS[workload]["bwd"])
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"].startswith(workload)
