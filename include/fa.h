@@ -198,8 +198,8 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
  * allocator has reserved most of the memory).
  *
  * Same arguments and results as fa_bwd, minus the workspace.  The scratch the
- * backward needs (fa_bwd_workspace_bytes(B, H, N, d) bytes: one fp32 per row
- * and an fp32 dQ accumulator) comes from one array of
+ * backward needs (fa_bwd_workspace_bytes(B, H, N, d) bytes: two fp32 per-row
+ * statistics and an fp32 dQ accumulator) comes from one array of
  * FA_NOALLOC_SCRATCH_BYTES bytes that the library holds in device memory on
  * every GPU that loads it, until the process exits.  Problems that need more
  * are rejected with FA_ERR_SCRATCH_LIMIT before anything is launched.
