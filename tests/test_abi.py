@@ -1,7 +1,8 @@
 """The C ABI without a GPU: the library loads, exports every function that
 include/fa.h declares, names every status, and rejects bad arguments with the
 documented status before any CUDA call (no pointer is dereferenced; the fake
-device addresses below are never touched)."""
+device addresses below are never touched).  The header is plain C99, and a C
+program linked against the library calls it."""
 import ctypes
 import os
 import re
@@ -169,3 +170,43 @@ def test_profile_read_rejects_null():
     lib = fa.load_library()
     assert lib.fa_profile_read(None, None) == INVALID
     assert lib.fa_version() >= 100
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "fa.h"
+
+int main(void) {
+    /* calls that need no GPU: the version, a status name, a workspace size,
+       and an argument check that returns before any CUDA call */
+    int rc = fa_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 128, 64, 0.125f, 0, FA_BF16, NULL);
+    size_t ws = fa_bwd_workspace_bytes(1, 1, 128, 64);
+    printf("%d %d %s %zu\n", fa_version(), rc, fa_status_string(FA_ERR_WORKSPACE), ws);
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_callable_from_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99, and a C program
+    # linked against the library calls it
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(fa.library_path())
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lfa_b200",
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    version, rc, *rest = out.stdout.split()
+    assert int(version) == fa.load_library().fa_version()
+    assert int(rc) == INVALID
+    assert int(rest[-1]) == fa.fa_bwd_workspace_bytes(1, 1, 128, 64) > 0
+    assert " ".join(rest[:-1]) == fa.fa_status_string(WORKSPACE)
