@@ -123,9 +123,14 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _on_device(t):
-    """Is t in device memory of the current device (where the library launches)?"""
-    return t.is_cuda and t.device.index == torch.cuda.current_device()
+def _current_device():
+    """Index of the current CUDA device, where the library launches (asked once per call)."""
+    return torch.cuda.current_device()
+
+
+def _on_device(t, dev):
+    """Is t in the memory of CUDA device dev?"""
+    return t.is_cuda and t.get_device() == dev
 
 
 _HALF = (torch.float16, torch.bfloat16)
@@ -133,14 +138,14 @@ _F32 = (torch.float32,)
 _U8 = (torch.uint8,)
 
 
-def _need(name, t, dtypes=None, shape=None, numel=None):
+def _need(name, t, dev, dtypes=None, shape=None, numel=None):
     """Checks one tensor argument before its address goes to the library, which
     cannot check a pointer: a contiguous tensor in the current device's memory,
     of an accepted dtype and of the given shape (or element count).  Raises
     TypeError / ValueError; nothing is launched."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
-    if not _on_device(t):
+    if not _on_device(t, dev):
         raise ValueError(f"{name}: must be a CUDA tensor on the current device (got {t.device})")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
@@ -155,24 +160,25 @@ def _need(name, t, dtypes=None, shape=None, numel=None):
 def _need_attention(q, k, v, o, lse, square, dout=None, dq=None, dk=None, dv=None, workspace=None,
                     block_mask=None, alibi_slopes=None):
     """Checks the tensors of one attention call; returns (B, H, Nq, Nk, d)."""
-    _need("q", q, _HALF)
+    dev = _current_device() if isinstance(q, torch.Tensor) and q.is_cuda else -1
+    _need("q", q, dev, _HALF)
     B, H, Nq, d = _shape(q)
-    _need("k", k, (q.dtype,))
+    _need("k", k, dev, (q.dtype,))
     if k.dim() != 4 or tuple(k.shape[:2]) != (B, H) or int(k.shape[3]) != d or (square and k.shape[2] != Nq):
         raise ValueError(f"k: shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
     Nk = int(k.shape[2])
-    _need("v", v, (q.dtype,), shape=k.shape)
-    _need("o", o, (q.dtype,), shape=q.shape)
-    _need("lse", lse, _F32, numel=B * H * Nq)
+    _need("v", v, dev, (q.dtype,), shape=k.shape)
+    _need("o", o, dev, (q.dtype,), shape=q.shape)
+    _need("lse", lse, dev, _F32, numel=B * H * Nq)
     for name, t, like in (("dout", dout, q), ("dq", dq, q), ("dk", dk, k), ("dv", dv, k)):
         if t is not None:
-            _need(name, t, (q.dtype,), shape=like.shape)
+            _need(name, t, dev, (q.dtype,), shape=like.shape)
     if workspace is not None:
-        _need("workspace", workspace)          # its size is the library's check
+        _need("workspace", workspace, dev)          # its size is the library's check
     if block_mask is not None:
-        _need("block_mask", block_mask, _U8, numel=((Nq + 127) // 128) * ((Nk + 127) // 128))
+        _need("block_mask", block_mask, dev, _U8, numel=((Nq + 127) // 128) * ((Nk + 127) // 128))
     if alibi_slopes is not None:
-        _need("alibi_slopes", alibi_slopes, _F32, numel=H)
+        _need("alibi_slopes", alibi_slopes, dev, _F32, numel=H)
     return B, H, Nq, Nk, d
 
 
@@ -343,12 +349,13 @@ def fa_fp8_quantize_qkv(q, k, v, signs=None, stream=None):
     """E4M3 codes and scales of q, k, v [B, H, N, d] (16-bit, on the device):
     returns (q8, k8, v8 uint8 [B, H, N, d], sq, sk, sv fp32 [B, H, ceil(N / 128)]).
     signs (fp32 [d] of +-1 on the device) rotates Q and K by diag(signs) H_d / sqrt(d)."""
-    _need("q", q, _HALF)
+    dev = _current_device() if isinstance(q, torch.Tensor) and q.is_cuda else -1
+    _need("q", q, dev, _HALF)
     B, H, N, d = _shape(q)
-    _need("k", k, (q.dtype,), shape=q.shape)
-    _need("v", v, (q.dtype,), shape=q.shape)
+    _need("k", k, dev, (q.dtype,), shape=q.shape)
+    _need("v", v, dev, (q.dtype,), shape=q.shape)
     if signs is not None:
-        _need("signs", signs, _F32, numel=d)
+        _need("signs", signs, dev, _F32, numel=d)
     nb = (N + 127) // 128
     q8, k8, v8 = (torch.empty((B, H, N, d), dtype=torch.uint8, device=q.device) for _ in range(3))
     sq, sk, sv = (torch.empty((B, H, nb), dtype=torch.float32, device=q.device) for _ in range(3))
@@ -361,15 +368,16 @@ def fa_fp8_quantize_qkv(q, k, v, signs=None, stream=None):
 def fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal=False, scale=None, stream=None):
     """FP8 forward on the codes and scales of fa_fp8_quantize_qkv; o [B, H, N, d]
     (float16 or bfloat16) and lse [B, H, N] fp32 are written."""
-    _need("q8", q8, _U8)
+    dev = _current_device() if isinstance(q8, torch.Tensor) and q8.is_cuda else -1
+    _need("q8", q8, dev, _U8)
     B, H, N, d = _shape(q8)
     nb = (N + 127) // 128
     for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
-        _need(name, t, _U8, shape=q8.shape)
+        _need(name, t, dev, _U8, shape=q8.shape)
     for name, t in (("sq", sq), ("sk", sk), ("sv", sv)):
-        _need(name, t, _F32, numel=B * H * nb)
-    _need("o", o, _HALF, shape=q8.shape)
-    _need("lse", lse, _F32, numel=B * H * N)
+        _need(name, t, dev, _F32, numel=B * H * nb)
+    _need("o", o, dev, _HALF, shape=q8.shape)
+    _need("lse", lse, dev, _F32, numel=B * H * N)
     rc = load_library().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o), _ptr(lse),
                                    B, H, N, d, _scale(scale, d), int(bool(causal)), _dtype(o), _stream(stream))
     _check(rc, "fa_fwd_fp8")

@@ -42,7 +42,8 @@ class _FakeLib:
 def fake(monkeypatch):
     lib = _FakeLib()
     monkeypatch.setattr(fa, "load_library", lambda: lib)
-    monkeypatch.setattr(fa, "_on_device", lambda t: True)
+    monkeypatch.setattr(fa, "_on_device", lambda t, dev: True)
+    monkeypatch.setattr(fa, "_current_device", lambda: 0)
     return lib
 
 
