@@ -208,3 +208,37 @@ def test_quantizer_matches_numpy_and_torch_float8():
             y = (blk * (np.float32(448.0) / amax)).astype(np.float32)
             ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
             assert np.array_equal(codes[h, b * 128:(b + 1) * 128], ref)
+
+
+@pytest.mark.parametrize("k_values", [(0.0, -1.0), (2.0, 1.0)])
+def test_fp8_rounded_p_hand_worked(k_values):
+    """A hand-worked case of reading 25 ("FlashAttention 深度解析" section 四:
+    FP8 block quantisation; P goes through E4M3 before P V): the scores of one
+    query against two keys differ by 1, so P = (1, e^-1) relative to the row
+    maximum.  On the E4M3 grid, e^-1 = 0.3679 lies between 1.375 * 2^-2 and
+    1.5 * 2^-2, above their midpoint 0.359375, so it rounds to 0.375.  With V
+    rows (1, 0) the output is 1 / (1 + 0.375) = 8/11, normalised by the sum of
+    the rounded P; LSE keeps the exact sum, max + ln(1 + e^-1).  The second
+    case shifts both scores by +2: P is taken relative to the maximum, so O is
+    unchanged (rounding e^2 and e^1 themselves would give 7.5 / 10.25)."""
+    code = {0.0: 0x00, 1.0: 0x38, -1.0: 0xB8, 2.0: 0x40}   # E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits
+    d = 16
+    q8 = np.zeros((1, 2, d), np.uint8)
+    q8[0, :, 0] = code[1.0]
+    k8 = np.zeros((1, 2, d), np.uint8)
+    k8[0, 0, 0], k8[0, 1, 0] = code[k_values[0]], code[k_values[1]]
+    v8 = np.zeros((1, 2, d), np.uint8)
+    v8[0, 0, 0] = code[1.0]
+    ones = np.ones((1, 1), np.float32)
+    o, lse = oracle.fwd_fp8(q8, k8, v8, ones, ones, np.ones(1, np.float32), 1.0)
+    want = np.zeros((2, d))
+    want[:, 0] = 8.0 / 11.0
+    assert np.allclose(o[0], want, rtol=0, atol=1e-15)
+    assert np.allclose(lse[0], k_values[0] + np.log1p(np.exp(-1.0)), rtol=0, atol=1e-15)
+    # causal: the first query sees only the first key, P = (1), O = v_0 = (1, 0, ...)
+    o, lse = oracle.fwd_fp8(q8, k8, v8, ones, ones, np.ones(1, np.float32), 1.0, causal=True)
+    assert o[0, 0, 0] == 1.0 and np.all(o[0, 0, 1:] == 0) and lse[0, 0] == k_values[0]
+    assert np.isclose(o[0, 1, 0], 8.0 / 11.0, rtol=0, atol=1e-15)
+    # without the rounding of P: 1 / (1 + e^-1)
+    o, _ = oracle.fwd_fp8(q8, k8, v8, ones, ones, np.ones(1, np.float32), 1.0, quant_p=False)
+    assert np.isclose(o[0, 0, 0], 1.0 / (1.0 + np.exp(-1.0)), rtol=0, atol=1e-15)

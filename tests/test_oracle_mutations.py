@@ -35,6 +35,17 @@ MUTANTS = {
     "alibi_offset_dropped": ("const double dist = fabs((double)i + ((double)sp->Nk - sp->Nq) - (double)j);",
                              "const double dist = fabs((double)i - (double)j);"),
     "alibi_head_ignored": ("return -sp->slopes[h % sp->H] * dist;", "return -sp->slopes[0] * dist;"),
+    # the remaining products and statistics of the definition, the online recurrence, the sampled path
+    "dq_scale_dropped": ("dq[(size_t)i * d + x] = c->scale * acc;", "dq[(size_t)i * d + x] = acc;"),
+    "delta_dropped": ("D[i] = acc;", "D[i] = 0.0;"),
+    "o_wrong_value_row": ("acc += P[(size_t)i * Nk + j] * v[(size_t)j * d + x];",
+                          "acc += P[(size_t)i * Nk + j] * v[(size_t)(Nk - 1 - j) * d + x];"),
+    "p_normalisation_dropped": ("for (int j = 0; j < N; ++j) srow[j] = exp(srow[j] - lse);",
+                                "for (int j = 0; j < N; ++j) srow[j] = exp(srow[j] - m);"),
+    "online_sum_rescale_dropped": ("            l *= corr;\n", ""),
+    "sampled_cols_wrong_lse_row": ("double p = exp(c->scale * s + bias(&c->sp, h, i, j) - lse[i]);",
+                                   "double p = exp(c->scale * s + bias(&c->sp, h, i, j) - lse[0]);"),
+    "sampled_cols_dv_uses_ds": ("dvj[x] += p * dout", "dvj[x] += ds * dout"),
 }
 
 # FP8 forward (E4M3, rotation, block quantiser, FP8 attention): checked by its own pins
@@ -46,6 +57,13 @@ FP8_MUTANTS = {
                                  "const float inv = amax > 0.0f ? amax / 448.0f : 1.0f;"),
     "fp8_v_scale_dropped": ("const double f = (double)c->sv[h] / l8;", "const double f = 1.0 / l8;"),
     "fp8_key_scale_uses_query_block": ("(double)c->sk[h * nb + j / c->rows]", "(double)c->sk[h * nb + i / c->rows]"),
+    "rotation_normalisation_dropped": ("for (int c = 0; c < d; ++c) x[c] = x[c] * r;", ""),
+    "fp8_p_left_unrounded": ("p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(pj)) : pj;", "p8[j] = pj;"),
+    "fp8_o_normalised_by_unrounded_sum": ("const double f = (double)c->sv[h] / l8;",
+                                          "const double f = (double)c->sv[h] / l;"),
+    "fp8_p_rounded_before_the_max": (
+        "p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(pj)) : pj;",
+        "p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(exp(s[j]))) * exp(-m) : pj;"),
 }
 
 PIN_FILES = ["test_oracle_pins.py", "test_oracle_modes.py"]
