@@ -46,6 +46,10 @@ MUTANTS = {
     "sampled_cols_wrong_lse_row": ("double p = exp(c->scale * s + bias(&c->sp, h, i, j) - lse[i]);",
                                    "double p = exp(c->scale * s + bias(&c->sp, h, i, j) - lse[0]);"),
     "sampled_cols_dv_uses_ds": ("dvj[x] += p * dout", "dvj[x] += ds * dout"),
+    "sampled_rows_ds_sign_flipped": ("double ds = prow[j] * (dp - D);", "double ds = prow[j] * (D - dp);"),
+    "sampled_rows_dq_scale_dropped": ("for (int x = 0; x < d; ++x) dqi[x] *= c->scale;", ""),
+    "empty_row_made_uniform": ("for (int j = 0; j < N; ++j) srow[j] = 0.0;",
+                               "for (int j = 0; j < N; ++j) srow[j] = 1.0 / N;"),
 }
 
 # FP8 forward (E4M3, rotation, block quantiser, FP8 attention): checked by its own pins
