@@ -65,6 +65,10 @@ FP8_MUTANTS = {
     "fp8_p_left_unrounded": ("p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(pj)) : pj;", "p8[j] = pj;"),
     "fp8_o_normalised_by_unrounded_sum": ("const double f = (double)c->sv[h] / l8;",
                                           "const double f = (double)c->sv[h] / l;"),
+    "quantiser_amax_of_first_row_only": ("for (size_t e = 0; e < n; ++e) amax = fmaxf(amax, fabsf(t[e]));",
+                                         "for (size_t e = 0; e < (size_t)d; ++e) amax = fmaxf(amax, fabsf(t[e]));"),
+    "e4m3_overflow_to_nan": ("if (a >= 448.0) return s | 0x7e;", "if (a >= 448.0) return s | 0x7f;"),
+    "rotation_signs_not_applied": ("for (int c = 0; c < d; ++c) x[c] = x[c] * signs[c];", ""),
     "fp8_p_rounded_before_the_max": (
         "p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(pj)) : pj;",
         "p8[j] = c->quant_p ? oracle_e4m3_value(oracle_e4m3_round(exp(s[j]))) * exp(-m) : pj;"),
