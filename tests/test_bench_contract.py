@@ -52,7 +52,7 @@ def test_peak_follows_the_sampled_clock():
 def test_every_workload_describes_itself_and_counts_flops(name):
     w = bench.WORKLOADS[name]
     assert bench.describe(name, w).startswith(name + ":")
-    kept = 52875 if w["sparse"] else None
+    kept = 52834 if w["sparse"] else None
     fwd, bwd = bench.workload_flops(w, kept)
     assert fwd > 0
     assert bwd == (2.5 * fwd if w["bwd"] else 0.0)
