@@ -380,6 +380,64 @@ def make_inputs_cpu(w):
     return dict(q=q, k=k, v=v, do=do, mask=mask, slopes=slopes), None
 
 
+def analyse(prof, w, name, fwd_f, bwd_f, clocks, steps):
+    """From the library's per-kernel CUDA-event times ({kind: (ms summed over
+    the timed steps, launches)}): the roofline of the dominant kernel, the
+    per-kernel table and the forward / backward split.  fwd_f, bwd_f: the
+    algorithmic FLOPs of one step's forward and backward."""
+    dom = max(prof, key=lambda k: prof[k][0])
+    dom_ms, dom_n = prof[dom]
+    per_launch_ms = dom_ms / max(dom_n, 1)
+    burst, sustained, hbm, src = peaks()
+    # a run that hit the power cap is compared with the sustained GEMM figure
+    # (cuBLAS under the same cap), a short one with the burst figure
+    capped = power_capped(clocks)
+    peak = sustained if capped and sustained else burst
+    peak_kind = "sustained (power-capped run)" if capped and sustained else "burst"
+    if dom == "fwd_fp8":
+        # an E4M3 contraction: the measured bf16 GEMM peak x the nominal fp8 : bf16 ratio (2)
+        achieved = fwd_f / (per_launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": 2 * peak, "unit": "TFLOP/s",
+                "frac": achieved / (2 * peak),
+                "peak_source": f"{src} bf16 {peak_kind} (MEASURED_PEAKS.json) x 2, the nominal fp8 : bf16 ratio",
+                "kernel": dom, "launch_ms": per_launch_ms}
+    elif dom == "fp8_quant":
+        # three launches per step: read Q, K, V and V again (16-bit), write three E4M3 tensors
+        n = w["B"] * w["H"] * w["N"] * w["d"]
+        alg_bytes = 4 * 2 * n + 3 * n
+        step_ms = dom_ms / steps
+        achieved = alg_bytes / (step_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "kernel": dom, "step_ms": step_ms, "algorithmic_bytes": alg_bytes}
+    elif dom in ("fwd", "bwd_main", "bwd_dq"):
+        # tensor FLOPs the kernel performs: the backward's five products, of
+        # which the deterministic backward's key-block kernel does four (no dQ)
+        # and its dQ pass three (S and dP again, then dQ)
+        det = w.get("deterministic", False)
+        alg = {"fwd": fwd_f, "bwd_main": bwd_f * (0.8 if det else 1.0), "bwd_dq": bwd_f * 0.6}[dom]
+        achieved = alg / (per_launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
+                "kernel": dom, "launch_ms": per_launch_ms}
+    else:
+        roof = {"bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None, "kernel": dom}
+    roof["traffic"] = traffic_for(dom, name)
+    total = max(sum(x[0] for x in prof.values()), 1e-12)
+    kernel_times = {k: {"ms_per_launch": (v[0] / v[1] if v[1] else 0.0), "launches": v[1], "share": v[0] / total}
+                    for k, v in prof.items()}
+    fkind = "fwd_fp8" if w.get("fp8") else "fwd"
+    fwd_ms = prof[fkind][0] / max(prof[fkind][1], 1)
+    fpeak = 2 * peak if w.get("fp8") else peak   # E4M3 products: twice the bf16 rate (nominal ratio)
+    split = {"fwd_tflops": fwd_f / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
+             "fwd_frac_of_peak": (fwd_f / (fwd_ms / 1e3) / 1e12) / fpeak if fwd_ms else None,
+             "peak": fpeak, "peak_kind": peak_kind}
+    if w["bwd"]:
+        bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post", "bwd_dq")) / max(prof["bwd_main"][1], 1)
+        split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12
+        split["bwd_frac_of_peak"] = split["bwd_tflops"] / peak
+    return roof, kernel_times, split
+
+
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
@@ -445,57 +503,8 @@ def run_ours(args, w, name):
     if fa.fa_last_device_status() != 0:
         raise RuntimeError("device status after the timed region is not ok")
 
-    # ---------------- dominant kernel roofline
-    dom = max(prof, key=lambda k: prof[k][0])
-    dom_ms, dom_n = prof[dom]
-    per_launch_ms = dom_ms / max(dom_n, 1)
-    burst, sustained, hbm, src = peaks()
-    # a run that hit the power cap is compared with the sustained GEMM figure
-    # (cuBLAS under the same cap), a short one with the burst figure
-    capped = power_capped(clocks)
-    peak = sustained if capped and sustained else burst
-    peak_kind = "sustained (power-capped run)" if capped and sustained else "burst"
-    if dom == "fwd_fp8":
-        # an E4M3 contraction: the measured bf16 GEMM peak x the nominal fp8 : bf16 ratio (2)
-        achieved = fwd_f / (per_launch_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": 2 * peak, "unit": "TFLOP/s",
-                "frac": achieved / (2 * peak),
-                "peak_source": f"{src} bf16 {peak_kind} (MEASURED_PEAKS.json) x 2, the nominal fp8 : bf16 ratio",
-                "kernel": dom, "launch_ms": per_launch_ms}
-    elif dom == "fp8_quant":
-        # three launches per step: read Q, K, V and V again (16-bit), write three E4M3 tensors
-        n = w["B"] * w["H"] * w["N"] * w["d"]
-        alg_bytes = 4 * 2 * n + 3 * n
-        step_ms = dom_ms / args.steps
-        achieved = alg_bytes / (step_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "kernel": dom, "step_ms": step_ms, "algorithmic_bytes": alg_bytes}
-    elif dom in ("fwd", "bwd_main", "bwd_dq"):
-        # tensor FLOPs the kernel performs: the backward's five products, of
-        # which the deterministic backward's key-block kernel does four (no dQ)
-        # and its dQ pass three (S and dP again, then dQ)
-        det = w.get("deterministic", False)
-        alg = {"fwd": fwd_f, "bwd_main": bwd_f * (0.8 if det else 1.0), "bwd_dq": bwd_f * 0.6}[dom]
-        achieved = alg / (per_launch_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{src} bf16 {peak_kind} (MEASURED_PEAKS.json)",
-                "kernel": dom, "launch_ms": per_launch_ms}
-    else:
-        alg_bytes = None
-        roof = {"bound": "hbm", "achieved": alg_bytes, "peak": hbm, "unit": "GB/s", "frac": None, "kernel": dom}
-    roof["traffic"] = traffic_for(dom, name)
-    kernel_times = {k: {"ms_per_launch": (v[0] / v[1] if v[1] else 0.0), "launches": v[1],
-                        "share": v[0] / max(sum(x[0] for x in prof.values()), 1e-12)} for k, v in prof.items()}
-    fkind = "fwd_fp8" if w.get("fp8") else "fwd"
-    fwd_ms = prof[fkind][0] / max(prof[fkind][1], 1)
-    fpeak = 2 * peak if w.get("fp8") else peak   # E4M3 products: twice the bf16 rate (nominal ratio)
-    split = {"fwd_tflops": fwd_f / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
-             "fwd_frac_of_peak": (fwd_f / (fwd_ms / 1e3) / 1e12) / fpeak if fwd_ms else None,
-             "peak": fpeak, "peak_kind": peak_kind}
-    if w["bwd"]:
-        bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post", "bwd_dq")) / max(prof["bwd_main"][1], 1)
-        split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12
-        split["bwd_frac_of_peak"] = split["bwd_tflops"] / peak
+    # ---------------- dominant kernel roofline, per-kernel times, forward/backward split
+    roof, kernel_times, split = analyse(prof, w, name, fwd_f, bwd_f, clocks, args.steps)
 
     # ---------------- the same steps replayed from a CUDA graph (launch overhead removed)
     graph = None

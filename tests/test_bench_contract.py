@@ -56,3 +56,56 @@ def test_every_workload_describes_itself_and_counts_flops(name):
     fwd, bwd = bench.workload_flops(w, kept)
     assert fwd > 0
     assert bwd == (2.5 * fwd if w["bwd"] else 0.0)
+
+
+def _prof(**ms_per_launch):
+    # {kind: (ms summed over 10 steps, launches)} as the library reports it
+    kinds = ("fwd", "bwd_pre", "bwd_main", "bwd_post", "bwd_dq", "fp8_quant", "fwd_fp8")
+    launches = {"fp8_quant": 30}
+    return {k: (ms_per_launch.get(k, 0.0) * launches.get(k, 10), launches.get(k, 10) if k in ms_per_launch else 0)
+            for k in kinds}
+
+
+FULL_CLOCK = {"sm_mhz": 1965.0, "sm_min_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+
+
+def test_analyse_the_dsweep128_step():
+    # per-launch times of the d = 128 sweep on one B200: forward 0.289 ms, backward main 0.772 ms
+    w = bench.WORKLOADS["dsweep128"]
+    fwd_f, bwd_f = bench.workload_flops(w)
+    prof = _prof(fwd=0.289, bwd_pre=0.03, bwd_main=0.772, bwd_post=0.02)
+    roof, kernels, split = bench.analyse(prof, w, "dsweep128", fwd_f, bwd_f, FULL_CLOCK, 10)
+    burst = bench.peaks()[0]
+    assert roof["kernel"] == "bwd_main" and roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert abs(roof["achieved"] - bwd_f / 0.772e-3 / 1e12) < 1e-6 and abs(roof["achieved"] - 890.3) < 1.0
+    assert roof["peak"] == burst and abs(roof["frac"] - roof["achieved"] / burst) < 1e-12
+    assert abs(split["fwd_tflops"] - 951.0) < 1.0
+    assert abs(split["bwd_tflops"] - bwd_f / 0.822e-3 / 1e12) < 1e-6
+    assert abs(sum(k["share"] for k in kernels.values()) - 1.0) < 1e-9
+    assert kernels["bwd_main"]["launches"] == 10 and abs(kernels["bwd_main"]["ms_per_launch"] - 0.772) < 1e-12
+    # a power-capped run (SM clock held below 95 % of max) is compared with the sustained figure
+    capped = dict(FULL_CLOCK, sm_mhz=1500.0, sm_min_mhz=1400.0, reasons=["sw_power_cap"])
+    roof2, _, split2 = bench.analyse(prof, w, "dsweep128", fwd_f, bwd_f, capped, 10)
+    assert roof2["peak"] == bench.peaks()[1] and split2["peak_kind"].startswith("sustained")
+
+
+def test_analyse_deterministic_and_fp8_steps():
+    w = bench.WORKLOADS["det128"]
+    fwd_f, bwd_f = bench.workload_flops(w)
+    # the key-block kernel without dQ performs four of the five products, the dQ pass three
+    roof, _, _ = bench.analyse(_prof(fwd=0.3, bwd_pre=0.03, bwd_main=0.513, bwd_dq=0.394), w, "det128",
+                               fwd_f, bwd_f, FULL_CLOCK, 10)
+    assert roof["kernel"] == "bwd_main" and abs(roof["achieved"] - 0.8 * bwd_f / 0.513e-3 / 1e12) < 1e-6
+    roof, _, _ = bench.analyse(_prof(fwd=0.3, bwd_pre=0.03, bwd_main=0.3, bwd_dq=0.394), w, "det128",
+                               fwd_f, bwd_f, FULL_CLOCK, 10)
+    assert roof["kernel"] == "bwd_dq" and abs(roof["achieved"] - 0.6 * bwd_f / 0.394e-3 / 1e12) < 1e-6
+    # FP8: the forward against twice the bf16 peak; the quantiser (three launches a step) against HBM
+    w = bench.WORKLOADS["fp8_128"]
+    fwd_f, bwd_f = bench.workload_flops(w)
+    roof, _, split = bench.analyse(_prof(fwd_fp8=0.289, fp8_quant=0.04), w, "fp8_128", fwd_f, bwd_f, FULL_CLOCK, 10)
+    assert roof["kernel"] == "fwd_fp8" and roof["peak"] == 2 * bench.peaks()[0]
+    assert split["peak"] == 2 * bench.peaks()[0] and "bwd_tflops" not in split
+    roof, _, _ = bench.analyse(_prof(fwd_fp8=0.05, fp8_quant=0.1), w, "fp8_128", fwd_f, bwd_f, FULL_CLOCK, 10)
+    n = 4 * 16 * 4096 * 128
+    assert roof["kernel"] == "fp8_quant" and roof["unit"] == "GB/s"
+    assert abs(roof["achieved"] - 11 * n / (0.3e-3) / 1e9) < 1e-6     # 0.1 ms x 3 launches per step
