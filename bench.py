@@ -469,6 +469,8 @@ def run_ours(args, w, name):
     in_bytes = sum(x.numel() * x.element_size() for x in (t["q"], t["k"], t["v"]) + ((t["do"],) if w["bwd"] else ()))
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device) if in_bytes <= L2_BYTES else None
     sampler = ClockSampler(local)
+    torch.cuda.reset_peak_memory_stats(device)
+    base_bytes = torch.cuda.memory_allocated(device)
     fa.fa_profile_enable(True)
     fa.fa_profile_read()
     fdist.barrier(device)
@@ -498,6 +500,13 @@ def run_ours(args, w, name):
     prof = fa.fa_profile_read()
     fa.fa_profile_enable(False)
     ms = sum(a.elapsed_time(b) for a, b in pairs)
+    # device memory: what the steps held (inputs, outputs, workspace) against
+    # one materialised N x N score matrix of the standard method
+    from flash_fwd_b200 import accounting as acc
+    memory = {"peak_allocated_bytes": torch.cuda.max_memory_allocated(device),
+              "allocated_before_steps_bytes": base_bytes,
+              "one_materialised_s_bytes": acc.s_matrix_bytes(w["B"], w["H"], w["N"], 2) * w.get("Nk", w["N"])
+              // w["N"]}
     ms_max = fdist.max_over_ranks(ms, device if args.gpus > 1 else None)
     value = fdist.aggregate_throughput([flops * args.steps] * world, ms_max) / 1e12
     if fa.fa_last_device_status() != 0:
@@ -594,6 +603,7 @@ def run_ours(args, w, name):
         "graph": graph,
         "device": device_info(local),
         "gpu_launches": sum(v[1] for v in prof.values()),
+        "memory": memory,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
