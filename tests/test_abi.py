@@ -210,3 +210,26 @@ def test_header_is_plain_c_and_callable_from_c(tmp_path):
     assert int(rc) == INVALID
     assert int(rest[-1]) == fa.fa_bwd_workspace_bytes(1, 1, 128, 64) > 0
     assert " ".join(rest[:-1]) == fa.fa_status_string(WORKSPACE)
+
+
+def test_every_entry_point_is_documented():
+    # a comment directly above each declaration, or the function named in a comment block
+    src = open(HEADER).read()
+    comments = " ".join(re.findall(r"/\*.*?\*/", src, flags=re.S))
+    lines = src.split("\n")
+    for i, line in enumerate(lines):
+        m = re.match(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", line)
+        if m:
+            above = "\n".join(lines[max(0, i - 3):i])
+            assert "*/" in above or m.group(1) in comments, m.group(1)
+
+
+def test_readme_names_real_workloads():
+    import bench
+    readme = open(os.path.join(ROOT, "README.md")).read()
+    for name in re.findall(r"--workload ([a-z0-9_]+)", readme):
+        assert name in bench.WORKLOADS, name
+    for name in re.findall(r"also: ([a-z0-9_, /]+)", readme):
+        for part in re.split(r"[ ,/]+", name):
+            if part and part[0].isalpha() and not part.startswith("also"):
+                assert part in bench.WORKLOADS or part.startswith("dsweep"), part
