@@ -380,6 +380,18 @@ def make_inputs_cpu(w):
     return dict(q=q, k=k, v=v, do=do, mask=mask, slopes=slopes), None
 
 
+SFU_EX2_PER_CLK_PER_SM = 16      # special-function unit, measured on B200 (one CTA per SM)
+SMS = 148
+
+
+def exp_ceiling_tflops(d, clocks):
+    """The forward's ceiling set by the exponential: one ex2 per score, each
+    score worth 4 d tensor FLOPs (S and P V), at the sampled SM clock (the
+    maximum when none was sampled)."""
+    mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz") or 1965.0
+    return SFU_EX2_PER_CLK_PER_SM * SMS * mhz * 1e6 * 4 * d / 1e12
+
+
 def analyse(prof, w, name, fwd_f, bwd_f, clocks, steps):
     """From the library's per-kernel CUDA-event times ({kind: (ms summed over
     the timed steps, launches)}): the roofline of the dominant kernel, the
@@ -421,6 +433,16 @@ def analyse(prof, w, name, fwd_f, bwd_f, clocks, steps):
                 "kernel": dom, "launch_ms": per_launch_ms}
     else:
         roof = {"bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None, "kernel": dom}
+    if dom in ("fwd", "fwd_fp8"):
+        # a forward is also bounded by its exponentials: where that ceiling is
+        # the lower one (d = 64; E4M3 products at d = 128) it is the roofline
+        ceiling = exp_ceiling_tflops(w["d"], clocks)
+        if ceiling < roof["peak"]:
+            roof.update({"bound": "alu", "tensor_peak": roof["peak"], "tensor_frac": roof["frac"],
+                         "tensor_peak_source": roof["peak_source"], "peak": ceiling,
+                         "frac": roof["achieved"] / ceiling,
+                         "peak_source": f"special-function unit: {SFU_EX2_PER_CLK_PER_SM} ex2 per clock per SM "
+                                        f"x {SMS} SMs x the sampled SM clock x 4 d FLOPs per ex2 (derived)"})
     roof["traffic"] = traffic_for(dom, name)
     total = max(sum(x[0] for x in prof.values()), 1e-12)
     kernel_times = {k: {"ms_per_launch": (v[0] / v[1] if v[1] else 0.0), "launches": v[1], "share": v[0] / total}
@@ -430,7 +452,7 @@ def analyse(prof, w, name, fwd_f, bwd_f, clocks, steps):
     fpeak = 2 * peak if w.get("fp8") else peak   # E4M3 products: twice the bf16 rate (nominal ratio)
     split = {"fwd_tflops": fwd_f / (fwd_ms / 1e3) / 1e12 if fwd_ms else None,
              "fwd_frac_of_peak": (fwd_f / (fwd_ms / 1e3) / 1e12) / fpeak if fwd_ms else None,
-             "peak": fpeak, "peak_kind": peak_kind}
+             "peak": fpeak, "peak_kind": peak_kind, "fwd_exp_ceiling": exp_ceiling_tflops(w["d"], clocks)}
     if w["bwd"]:
         bwd_ms = sum(prof[k][0] for k in ("bwd_pre", "bwd_main", "bwd_post", "bwd_dq")) / max(prof["bwd_main"][1], 1)
         split["bwd_tflops"] = bwd_f / (bwd_ms / 1e3) / 1e12

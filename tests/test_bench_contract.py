@@ -103,9 +103,29 @@ def test_analyse_deterministic_and_fp8_steps():
     w = bench.WORKLOADS["fp8_128"]
     fwd_f, bwd_f = bench.workload_flops(w)
     roof, _, split = bench.analyse(_prof(fwd_fp8=0.289, fp8_quant=0.04), w, "fp8_128", fwd_f, bwd_f, FULL_CLOCK, 10)
-    assert roof["kernel"] == "fwd_fp8" and roof["peak"] == 2 * bench.peaks()[0]
+    # at d = 128 the exponentials (512 FLOPs each, 16 per clock per SM) cap E4M3 attention below twice
+    # the bf16 rate: 16 x 148 x 1965 MHz x 512 = 2382 TFLOP/s
+    assert roof["kernel"] == "fwd_fp8" and roof["bound"] == "alu" and abs(roof["peak"] - 2382.4) < 0.5
+    assert roof["tensor_peak"] == 2 * bench.peaks()[0] and abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-12
     assert split["peak"] == 2 * bench.peaks()[0] and "bwd_tflops" not in split
     roof, _, _ = bench.analyse(_prof(fwd_fp8=0.05, fp8_quant=0.1), w, "fp8_128", fwd_f, bwd_f, FULL_CLOCK, 10)
     n = 4 * 16 * 4096 * 128
     assert roof["kernel"] == "fp8_quant" and roof["unit"] == "GB/s"
     assert abs(roof["achieved"] - 11 * n / (0.3e-3) / 1e9) < 1e-6     # 0.1 ms x 3 launches per step
+
+
+def test_forward_roofline_takes_the_lower_ceiling():
+    # d = 128 bf16: the exponential ceiling (2382) is above the tensor peak, which stays the roofline
+    w = bench.WORKLOADS["long_fwd"]
+    fwd_f, bwd_f = bench.workload_flops(w)
+    roof, _, _ = bench.analyse(_prof(fwd=0.25), w, "long_fwd", fwd_f, bwd_f, FULL_CLOCK, 10)
+    assert roof["bound"] == "tensor" and roof["peak"] == bench.peaks()[0] and "tensor_peak" not in roof
+    # d = 64: 256 FLOPs per exponential cap the forward at 1191 TFLOP/s, below the tensor peak
+    w = dict(bench.WORKLOADS["dsweep64"], bwd=False)
+    fwd_f, bwd_f = bench.workload_flops(w)
+    roof, _, split = bench.analyse(_prof(fwd=0.25), w, "dsweep64", fwd_f, bwd_f, FULL_CLOCK, 10)
+    assert roof["bound"] == "alu" and abs(roof["peak"] - 1191.2) < 0.5 and roof["tensor_peak"] == bench.peaks()[0]
+    assert abs(split["fwd_exp_ceiling"] - roof["peak"]) < 1e-9
+    # the ceiling follows the sampled SM clock
+    slow = dict(FULL_CLOCK, sm_mhz=1500.0)
+    assert abs(bench.exp_ceiling_tflops(64, slow) - 1191.2 * 1500 / 1965) < 0.5
