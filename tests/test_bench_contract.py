@@ -129,3 +129,18 @@ def test_forward_roofline_takes_the_lower_ceiling():
     # the ceiling follows the sampled SM clock
     slow = dict(FULL_CLOCK, sm_mhz=1500.0)
     assert abs(bench.exp_ceiling_tflops(64, slow) - 1191.2 * 1500 / 1965) < 0.5
+
+
+def test_clock_samples_are_summarised():
+    lines = ["0, 1965, 1965, 650.1, Not Active, Not Active, Not Active, Not Active",
+             "0, 1965, 1965, 998.0, Not Active, Not Active, Not Active, Active",
+             "0, 1800, 1965, 1001.3, Not Active, Not Active, Not Active, Active",
+             "0, [N/A], 1965, 10.0, Not Active, Not Active, Not Active, Not Active",   # unreadable: skipped
+             "garbage"]
+    c = bench.parse_clock_samples(lines)
+    assert c["samples"] == 3 and c["sm_mhz"] == 1965.0 and c["sm_min_mhz"] == 1800.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    assert bench.power_capped(c)           # a sample at 1800 MHz is below 95 % of 1965
+    hot = bench.parse_clock_samples(["0, 1400, 1965, 700, Active, Not Active, Active, Not Active"])
+    assert hot["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.parse_clock_samples([])["sm_mhz"] is None
