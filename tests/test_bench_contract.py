@@ -144,3 +144,20 @@ def test_clock_samples_are_summarised():
     hot = bench.parse_clock_samples(["0, 1400, 1965, 700, Active, Not Active, Active, Not Active"])
     assert hot["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.parse_clock_samples([])["sm_mhz"] is None
+
+
+def test_traffic_is_reported_only_for_unchanged_kernel_sources(tmp_path, monkeypatch):
+    import json as _json
+    sha = bench.kernel_source_sha()
+    assert len(sha) == 16
+    prof_dir = tmp_path / "profiles"
+    prof_dir.mkdir()
+    (prof_dir / "traffic.json").write_text(_json.dumps({
+        "fwd": {"dsweep128": {"bytes_per_launch": 123, "source_sha": sha}},
+        "bwd_main": {"dsweep128": {"bytes_per_launch": 456, "source_sha": "0" * 16}}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: sha)
+    assert bench.traffic_for("fwd", "dsweep128") == 123          # captured with these sources
+    assert bench.traffic_for("bwd_main", "dsweep128") is None    # sources changed since the capture
+    assert bench.traffic_for("fwd", "det128") is None            # never captured
+    assert bench.traffic_for("fwd_fp8", "fp8_128") is None
