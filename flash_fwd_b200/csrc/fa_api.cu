@@ -368,22 +368,14 @@ int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, vo
 // stand-in for the symbol, so the device address is looked up per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[kMaxDevices] = {};
-
-// The current device's address of g_noalloc_scratch, looked up on first use.
+// The current device's address of g_noalloc_scratch.  Looked up on every
+// call (a host-side table lookup once the module is loaded on the device), so
+// that no address outlives the context it belongs to: after a
+// cudaDeviceReset the module is loaded again and the array may move.
 int noalloc_scratch(void **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> g(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return FA_ERR_CUDA;
-        g_noalloc_addr[dev] = ptr;
-    }
-    *out = g_noalloc_addr[dev];
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return FA_ERR_CUDA;
+    *out = ptr;
     return FA_OK;
 }
 

@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(512, 1)
                     uint32_t sr[64];
                     tmem_ld32(tmem + lane_off + C::kColS + q0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                     tmem_ld32(tmem + lane_off + C::kColS + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                    tmem_ld_wait();
+                    tmem_wait_ld(sr);
                     if (GENERAL && p.alibi) {
                         // score + bias / scale, bias = -slope |q + off - key|
                         const float sl = -p.alibi[bh % p.H] / p.scale;
@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(512, 1)
                     uint32_t pr[64];
                     tmem_ld32(tmem + lane_off + C::kColDP + q0, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
                     tmem_ld32(tmem + lane_off + C::kColDP + q0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
-                    tmem_ld_wait();
+                    tmem_wait_ld(pr);
                     // row r of a K-major [128 keys][64 queries] 128B-swizzled tile
                     uint8_t *sdS = smem + C::kdSOff + qh * C::kChunk + r * 128;
 #pragma unroll
@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                 for (int ch = 0; ch < BM / 32; ++ch)
                     tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
-                tmem_ld_wait();
+                tmem_wait_ld(v);
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarDqFree));
                 if (row_lane) {

@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(352, 1)
                 uint32_t sr[64];
                 tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld_wait();
+                tmem_wait_ld(sr);
                 if (GENERAL && p.alibi) {
                     // score + bias / scale, bias = -slope |q + off - key|
                     const float base = static_cast<float>(rk);
@@ -463,13 +463,13 @@ __global__ void __launch_bounds__(352, 1)
                 uint32_t pr[32];
                 const uint32_t tP = tmem + lane_off + C::kColDP + 64 * kh;
                 tmem_ld32(tP, pr);
-                tmem_ld_wait();
+                tmem_wait_ld(pr);
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
                     ds[k] = pack2<BF16>(pv[2 * k] * (__uint_as_float(pr[2 * k]) - dd),
                                         pv[2 * k + 1] * (__uint_as_float(pr[2 * k + 1]) - dd));
                 tmem_ld32(tP + 32, pr);
-                tmem_ld_wait();
+                tmem_wait_ld(pr);
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarDPFree));
 #pragma unroll

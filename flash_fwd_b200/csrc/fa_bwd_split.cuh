@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(320, 1)
                 uint32_t sr[32], pr[32];
                 tmem_ld32(tmem + lane_off + C::kColS + 32 * ch, sr);
                 tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, pr);
-                tmem_ld_wait();
+                tmem_wait_ld(sr, pr);
                 if (GENERAL && p.alibi) {
                     // score + bias / scale, bias = -slope |q + off - key|
                     const float sl = -p.alibi[bh % p.H] / p.scale;

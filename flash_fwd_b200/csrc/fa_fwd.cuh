@@ -395,6 +395,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         const float c = p.scale_log2;
         float m = -INFINITY, l = 0.f, l_r = 0.f;
         int cnt = 0;
+        // does this row see any key?  Taken from the band limits of the tiles
+        // it meets, not from m or l: a row that sees no key keeps m = -inf
+        // only while every masked score stays -inf, and the polynomial exp2
+        // gives masked scores 2^-125 instead of 0
+        bool seen = false;
         KvIter<NQ, GENERAL> it;
         int j;
         uint32_t f;
@@ -409,7 +414,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
-            tmem_ld_wait();
+            tmem_wait_ld(r);
             // the scores as floats: a copy, not a float* view of r (reading
             // the asm-written integers through another type is undefined and
             // let stale register values into the row max)
@@ -428,6 +433,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 if ((p.mode & kCausal) && j == rb) hi = row_local;                    // diagonal tile
                 if (j == p.nkb - 1 && (p.Nk & 127)) hi = min(hi, (p.Nk & 127) - 1);  // key tail
             }
+            seen |= max(lo, 0) <= min(hi, 127);
             if (GENERAL && p.alibi) {
                 // score + bias / scale, bias = -slope |row + off - key|
                 const float sl = -p.alibi[bh % p.H] / p.scale;
@@ -538,9 +544,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         if (epi) {
             const bool valid = row < p.Nq;
             const float l_o = BF16 ? l_r : l;
-            // m = -inf: the row saw no key.  (The polynomial exp2 gives 2^-125,
-            // not 0, for masked scores, so l alone would not tell.)
-            const float inv_l = (cnt > 0 && l_o > 0.f && m != -INFINITY) ? 1.0f / l_o : 0.0f;
+            // a row that saw no key: O = 0, LSE = -inf
+            const float inv_l = (seen && l_o > 0.f) ? 1.0f / l_o : 0.0f;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
@@ -564,8 +569,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 }
             }
             if (valid) {
-                const float lse = (cnt > 0 && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f
-                                                        : -INFINITY;
+                const float lse = (seen && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
                 p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
             }
         }

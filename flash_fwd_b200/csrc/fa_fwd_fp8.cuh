@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
-            tmem_ld_wait();
+            tmem_wait_ld(r);
             // the scores as floats: a copy, not a float* view of r (reading
             // the asm-written integers through another type is undefined and
             // let stale register values into the row max)

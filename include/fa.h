@@ -204,8 +204,9 @@ FA_API int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const
  * every GPU that loads it, until the process exits.  Problems that need more
  * are rejected with FA_ERR_SCRATCH_LIMIT before anything is launched.
  *
- * The first call on a device looks up that device's address of the array
- * (cudaGetSymbolAddress, with the device current); make that first call
+ * Every call looks up the current device's address of the array
+ * (cudaGetSymbolAddress, with that device current); the first call on a
+ * device also loads the library's module there, so make that first call
  * before any stream capture.  Every call on a device shares the one array, so
  * calls whose kernels overlap on the GPU (different streams without ordering
  * between them) race and give wrong results; order them on one stream.  The

@@ -4,9 +4,12 @@ the C ABI binding) and -> fp64 oracle, compared element by element.
 Tolerances (max absolute error unless stated):
   O   1e-2 (fp16), 2e-2 (bf16)
   LSE 1e-3
-  dQ, dK, dV  5e-2 * max |oracle value| of that tensor, the max floored at
-              0.1: a tensor that is exactly zero in exact arithmetic (dQ and dK
-              at N = 1, where every row has one key) is held to 5e-3 absolute
+  dQ, dK, dV  5e-2 * max |oracle value| of that tensor.  Only a tensor whose
+              oracle values are all exactly zero (dQ and dK at N = 1, where
+              every row has one key) is held to 5e-3 absolute instead.  A
+              sampled check normalises by the largest oracle value among the
+              sampled elements, a lower bound of the tensor's maximum, so its
+              bar is never looser than the one on the whole tensor.
 """
 import numpy as np
 import torch
@@ -18,6 +21,12 @@ TOL_O = {"f16": 1e-2, "bf16": 2e-2}
 TOL_LSE = 1e-3
 TOL_GRAD_REL = 5e-2
 GRAD_NORM_FLOOR = 0.1
+
+
+def grad_norm(want_max):
+    """The normaliser of the gradient bar for an oracle tensor whose largest
+    magnitude is `want_max` (the floor applies only to an exactly zero tensor)."""
+    return want_max if want_max > 0.0 else GRAD_NORM_FLOOR
 
 
 def bh(x):
@@ -99,7 +108,7 @@ def check_bwd(grads_gpu, q, k, v, do, causal, scale, mask=None, dq_rows=None, kv
         _, _, rdq, rdk, rdv = oracle.bwd_full(Q, K, V, DO, scale, fl, mk)
         pairs = {"dq": (dq, rdq), "dk": (dk, rdk), "dv": (dv, rdv)}
         for name, (got, want) in pairs.items():
-            errs[name] = np.abs(got - want).max() / max(np.abs(want).max(), GRAD_NORM_FLOOR)
+            errs[name] = np.abs(got - want).max() / grad_norm(np.abs(want).max())
     else:
         hs = range(B * H) if heads is None else heads
         worst = {"dq": [0.0, 0.0], "dk": [0.0, 0.0], "dv": [0.0, 0.0]}
@@ -117,7 +126,53 @@ def check_bwd(grads_gpu, q, k, v, do, causal, scale, mask=None, dq_rows=None, kv
                                     ("dv", dv[hh, cols], rdv[0])):
                 worst[name][0] = max(worst[name][0], np.abs(got - want).max())
                 worst[name][1] = max(worst[name][1], np.abs(want).max())
-        errs = {n: e / max(m, GRAD_NORM_FLOOR) for n, (e, m) in worst.items()}
+        errs = {n: e / grad_norm(m) for n, (e, m) in worst.items()}
     for name, e in errs.items():
         assert e <= TOL_GRAD_REL, f"{name} relative max err {e}"
+    return errs
+
+
+def oracle_all(q, k, v, do, causal, scale, mask=None, with_bwd=True):
+    """The oracle's O, LSE and (with_bwd) dQ, dK, dV on every element.
+
+    The forward runs over every query row; the gradients come from the row
+    (dQ) and column (dK, dV) entry points over every row and every key, which
+    give the same values as the full materialising backward (pinned on CPU)
+    without its column-strided loops, so the workload shapes finish in
+    seconds to about a minute on the host cores.
+    """
+    Q, K, V = bh(q), bh(k), bh(v)
+    N = Q.shape[1]
+    fl, mk = flags(causal, mask), mask_np(mask)
+    ref = {}
+    ref["o"], ref["lse"] = oracle.fwd(Q, K, V, scale, fl, mk)
+    if with_bwd:
+        DO = bh(do)
+        every = np.arange(N, dtype=np.int32)
+        ref["dq"] = oracle.bwd_dq_rows(Q, K, V, DO, scale, every, fl, mk)
+        ref["dk"], ref["dv"] = oracle.bwd_dkdv_cols(Q, K, V, DO, scale, every, fl, mk)
+    return ref
+
+
+def compare_fwd(o_gpu, lse_gpu, ref, dtype):
+    """Max errors of O and LSE against oracle_all's result, asserted against the bars."""
+    og = o_gpu.reshape(ref["o"].shape).double().numpy()
+    lg = lse_gpu.reshape(ref["lse"].shape).double().numpy()
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    worst_o = np.abs(og - ref["o"]).max()
+    worst_l = np.abs(lg - ref["lse"]).max()
+    assert worst_o <= TOL_O[dtype], f"O max err {worst_o}"
+    assert worst_l <= TOL_LSE, f"LSE max err {worst_l}"
+    return worst_o, worst_l
+
+
+def compare_bwd(grads_gpu, ref):
+    """Relative max errors of dQ, dK, dV against oracle_all's result, asserted."""
+    errs = {}
+    for name, g in zip(("dq", "dk", "dv"), grads_gpu):
+        want = ref[name]
+        got = g.reshape(want.shape).double().numpy()
+        assert np.isfinite(got).all(), name
+        errs[name] = np.abs(got - want).max() / grad_norm(np.abs(want).max())
+        assert errs[name] <= TOL_GRAD_REL, f"{name} relative max err {errs[name]}"
     return errs

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from flash_fwd_b200 import inputs
-from parity import GRAD_NORM_FLOOR, TOL_GRAD_REL, check_bwd
+from parity import TOL_GRAD_REL, check_bwd, grad_norm
 
 pytestmark = pytest.mark.gpu
 
@@ -51,7 +51,7 @@ def _check(grads, q, k, v, do, causal, scale, window=None, slopes=None, mask=Non
     dq, dk, dv = grads
     for name, g, r in (("dq", f(dq, Nq), ref[2]), ("dk", f(dk, Nk), ref[3]), ("dv", f(dv, Nk), ref[4])):
         assert np.isfinite(g).all(), name
-        err = np.abs(g - r).max() / max(np.abs(r).max(), GRAD_NORM_FLOOR)
+        err = np.abs(g - r).max() / grad_norm(np.abs(r).max())
         assert err <= TOL_GRAD_REL, (name, err)
 
 
@@ -143,17 +143,7 @@ def test_det_bitwise_reproducible(d, causal):
     torch.cuda.synchronize()
     assert torch.equal(dk_a, runs[0][1]) and torch.equal(dv_a, runs[0][2])
     diff = (dq_a.float() - runs[0][0].float()).abs().max().item()
-    assert diff <= 2e-2 * max(dq_a.float().abs().max().item(), GRAD_NORM_FLOOR)
-
-
-@pytest.mark.parametrize("d", [64, 128, 256])
-def test_det_dsweep_config_sampled(d):
-    # the B=4 H=16 N=4096 causal workload, dQ rows and dK/dV keys sampled per head
-    c = inputs.CONFIGS["dsweep"]
-    q, k, v, do = inputs.make_qkv(c["B"], c["H"], c["N"], d, c["dtype"], seed=0)
-    scale = inputs.default_scale(d)
-    grads = _run(q, k, v, do, True, scale)
-    check_bwd(grads, q, k, v, do, True, scale, dq_rows=16, kv_cols=16, heads=[0, 17, 38, 63])
+    assert diff <= 2e-2 * grad_norm(dq_a.float().abs().max().item())
 
 
 def test_det_workspace_and_errors():

@@ -8,13 +8,13 @@ import torch
 
 import oracle
 from flash_fwd_b200 import inputs
-from parity import GRAD_NORM_FLOOR, TOL_GRAD_REL, TOL_LSE, TOL_O
+from parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_norm
 
 pytestmark = pytest.mark.gpu
 
 
 def _grads_close(got, want):
-    return np.abs(got - want).max() / max(np.abs(want).max(), GRAD_NORM_FLOOR) <= TOL_GRAD_REL
+    return np.abs(got - want).max() / grad_norm(np.abs(want).max()) <= TOL_GRAD_REL
 
 
 @pytest.mark.parametrize("deterministic", [False, True])
