@@ -9,28 +9,32 @@
 //
 // Three launches on the caller's stream:
 //   bwd_pre   D = rowsum(dO o O) into the workspace; zeroes the fp32 dQ accumulator.
-//   bwd_main  one CTA per 128-key block (x DSPLIT column halves for d = 256).  The
-//             CTA keeps K_j, V_j in shared memory and its dK, dV accumulators in
-//             tensor memory while it sweeps the kept query tiles Q_i, dO_i
-//             (BM rows each) through an NS-stage TMA ring:
+//   bwd_main  one CTA per 128-key block (bwd_kernel, d <= 128; the d = 256
+//             kernel of fa_bwd_split.cuh splits the block's columns over two
+//             CTAs).  The CTA keeps K_j, V_j in shared memory and its dK, dV
+//             accumulators in tensor memory while it sweeps the kept 128-row
+//             query tiles Q_i, dO_i through an NS-stage TMA ring:
 //               S^T  = K_j Q_i^T   and  dP^T = V_j dO_i^T   (tcgen05, TMEM)
-//               P^T, dS^T          (softmax-grad warps, one thread per key row,
-//                                   written as 16-bit swizzled tiles to smem)
-//               dV  += P^T dO_i,   dK += dS^T Q_i        (tcgen05, TMEM)
-//               dQ_i = dS K_j  (d = 64)  or  dQ_i^T = K_j^T dS^T  (d >= 128)
-//                                  (tcgen05, TMEM), then fp32 atomics into the
-//                                   accumulator by the drain warps.
+//               P^T  (16-bit, written back over S^T in TMEM)
+//               dS^T (16-bit swizzled tile in shared memory)
+//               dV  += P^T dO_i  (TS form),   dK += dS^T Q_i
+//               dQ_i^T = K_j^T dS^T  (M = d), into the dP^T columns once dP^T
+//                                   has been read, then fp32 reductions into
+//                                   the accumulator by the drain warps.
 //   bwd_post  dQ = scale * accumulator, rounded to the 16-bit type.
 // The deterministic backward passes a null accumulator: bwd_main then computes
-// dK, dV only, and the dQ pass of fa_bwd_dq.cuh replaces the atomics and
+// dK, dV only, and the dQ pass of fa_bwd_dq.cuh replaces the reductions and
 // bwd_post.
 //
-// Warp roles of bwd_main: warps 0-3 softmax-grad (and the dV epilogue), warps
-// 4-7 dQ drain (and the dK epilogue), warp 8 TMA producer (also stages the
-// per-row LSE and D of each query tile), warp 9 MMA issuer (owns TMEM).
-// TMEM columns: S^T [0, BM), dP^T [128, 128 + BM), dV [256, 256 + DH),
-// dK [256 + DH, 256 + 2 DH), dQ at [64, 128) (transposed form) or
-// [256 + 2 DH, 256 + 3 DH) (d = 64).
+// Warp roles of bwd_kernel (512 threads): warps 0-7 softmax-grad (warp w owns
+// TMEM lanes 32 (w mod 4) .. +31, i.e. those keys, for queries
+// [64 (w div 4), +64) of the tile) and the dV (warps 0-3) / dK (warps 4-7)
+// epilogue; warps 8-11 dQ drain; warp 12 TMA producer (also bulk-copies the
+// per-row LSE * log2 e and D of each query tile); warp 13 MMA issuer (owns
+// TMEM); warps 14-15 idle.
+// TMEM columns: S^T / P^T [0, 128), dP^T [128, 256) (then dQ^T: at d = 128
+// every lane is a d index, at d = 64 the M = 64 product puts row m in lane
+// 32 (m / 16) + m % 16), dV [256, 256 + d), dK [256 + d, 256 + 2 d).
 #pragma once
 
 #include "fa_common.cuh"

@@ -283,3 +283,45 @@ def fwd_fp8(q8, k8, v8, sq, sk, sv, scale, causal=False, rows=None, quant_p=True
                                _threads(nthreads))
     assert rc == 0, rc
     return o, lse
+
+
+def fp8_o_bounds(q8, k8, v8, sq, sk, sv, scale, causal, rows, o_ref, blk=128):
+    """Bars on |O_kernel - O_oracle| of FP8 attention for query `rows` of ONE
+    (batch, head): q8, k8, v8 uint8 [N, d], sq, sk float32 [ceil(N / blk)],
+    sv the head's V scale, o_ref the oracle's O on those rows.
+
+    Both sides round each P_j to E4M3 and divide by the sum of the rounded
+    values; they take the rounding on differently scaled P (the kernel relative
+    to its lazily rescaled running maximum, the oracle relative to the exact
+    maximum), so each error e_j is within the half step
+    u_j = max(2^-4 P_j, 2^-10) of P_j <= 1 (3 mantissa bits; the subnormal
+    step 2^-9).  With O_o the oracle's result,
+        O_k - O_o = sum_j (e_j - e'_j) (v_j - O_o) / sum_j (P_j + e_j),
+    so |O_k - O_o| <= sum_j 2 u_j |v_j - O_o| / (sum_j P_j - sum_j u_j).
+    Returns (worst, six_sigma): the worst case above, and 6 standard
+    deviations of the same sum with the e_j independent and uniform; each plus
+    the 16-bit rounding of the kernel's output and 1e-4 for its fp32 sums.
+    """
+    vals = e4m3_values()
+    N = q8.shape[0]
+    b = np.arange(N) // blk
+    Q = vals[q8] * np.asarray(sq, dtype=np.float64)[b][:, None]
+    K = vals[k8] * np.asarray(sk, dtype=np.float64)[b][:, None]
+    V = vals[v8] * float(sv)
+    rows = np.asarray(rows)
+    S = scale * Q[rows] @ K.T
+    if causal:
+        S = np.where(np.arange(N)[None, :] > rows[:, None], -np.inf, S)
+    P = np.exp(S - S.max(1, keepdims=True))
+    u = np.minimum(P, np.maximum(P * 2.0 ** -4, 2.0 ** -10))   # below 2^-10 the code may be 0: error P
+    den = P.sum(1, keepdims=True)
+    worst = np.empty_like(o_ref)
+    for r0 in range(0, len(rows), 32):                      # |v_j - O_o| for 32 rows at a time
+        dev = np.abs(V[None, :, :] - o_ref[r0:r0 + 32, None, :])
+        worst[r0:r0 + 32] = np.einsum("rn,rnd->rd", 2 * u[r0:r0 + 32], dev)
+    worst /= den - u.sum(1, keepdims=True)
+    w = (2 * u) ** 2 / 3.0
+    var = w @ (V ** 2) - 2 * (w @ V) * o_ref + w.sum(1, keepdims=True) * o_ref ** 2
+    sigma = np.sqrt(np.maximum(var, 0.0)) / den
+    tail = lambda x: x + 2.0 ** -8 * (np.abs(o_ref) + x) + 1e-4   # noqa: E731
+    return tail(worst), tail(6 * sigma)

@@ -223,13 +223,3 @@ def test_every_entry_point_is_documented():
             above = "\n".join(lines[max(0, i - 3):i])
             assert "*/" in above or m.group(1) in comments, m.group(1)
 
-
-def test_readme_names_real_workloads():
-    import bench
-    readme = open(os.path.join(ROOT, "README.md")).read()
-    for name in re.findall(r"--workload ([a-z0-9_]+)", readme):
-        assert name in bench.WORKLOADS, name
-    for name in re.findall(r"also: ([a-z0-9_, /]+)", readme):
-        for part in re.split(r"[ ,/]+", name):
-            if part and part[0].isalpha() and not part.startswith("also"):
-                assert part in bench.WORKLOADS or part.startswith("dsweep"), part

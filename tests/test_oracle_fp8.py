@@ -242,3 +242,42 @@ def test_fp8_rounded_p_hand_worked(k_values):
     # without the rounding of P: 1 / (1 + e^-1)
     o, _ = oracle.fwd_fp8(q8, k8, v8, ones, ones, np.ones(1, np.float32), 1.0, quant_p=False)
     assert np.isclose(o[0, 0, 0], 1.0 / (1.0 + np.exp(-1.0)), rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("scale", [0.125, 1.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_o_bound_covers_rounding_at_other_scales(causal, scale):
+    # The GPU rounds P to E4M3 relative to a running maximum that may sit up to
+    # 2^8 below the true one (lazy rescale), the oracle relative to the exact
+    # maximum.  Emulate the kernel's choice with a random scale 2^delta per row
+    # and key tile, delta in [0, 8], and check that both bars of
+    # oracle.fp8_o_bounds hold.  With diffuse attention (scale 0.125) the
+    # worst case is loose (every key below 2^-6 may carry the subnormal
+    # half-step 2^-10); with peaked attention (scale 1) it is a tight bar.
+    g = torch.Generator().manual_seed(11)
+    N, d = 300, 64
+    x = torch.randn((3, N, d), generator=g).numpy().astype(np.float32) * np.float32(2.5)
+    q8, sq = oracle.fp8_quantize(x[0:1], 128)
+    k8, sk = oracle.fp8_quantize(x[1:2], 128)
+    v8, sv = oracle.fp8_quantize(x[2:3], N)
+    o_ref, _ = oracle.fwd_fp8(q8, k8, v8, sq, sk, sv[:, 0], scale, causal=causal)
+    vals = oracle.e4m3_values()
+    b = np.arange(N) // 128
+    Q = vals[q8[0]] * sq[0][b][:, None].astype(np.float64)
+    K = vals[k8[0]] * sk[0][b][:, None].astype(np.float64)
+    V = vals[v8[0]] * float(sv[0, 0])
+    S = scale * Q @ K.T
+    if causal:
+        S = np.where(np.arange(N)[None, :] > np.arange(N)[:, None], -np.inf, S)
+    P = np.exp(S - S.max(1, keepdims=True))
+    rng = np.random.default_rng(5)
+    delta = rng.integers(0, 9, size=(N, (N + 127) // 128))[:, b]          # per row and key tile
+    Ph = vals[oracle.e4m3_round(P * 2.0 ** delta)] * 2.0 ** -delta.astype(np.float64)
+    o_emul = (Ph @ V) / Ph.sum(1, keepdims=True)
+    worst, six_sigma = oracle.fp8_o_bounds(q8[0], k8[0], v8[0], sq[0], sk[0], sv[0, 0], scale, causal,
+                                           np.arange(N), o_ref[0])
+    err = np.abs(o_emul - o_ref[0])
+    assert np.all(err <= worst), float((err / worst).max())
+    assert np.all(err <= six_sigma), float((err / six_sigma).max())
+    if scale == 1.0:
+        assert np.median(worst) < 0.02 * np.abs(V).max()
