@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -146,11 +147,23 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, GENERAL>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
-    const long long ctas = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
-    if (ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    const long long items = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
+    if (items > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    fa::FwdParams pp = p;
+    pp.nitems = static_cast<int>(items);
+    // two query tiles per item: one resident CTA per SM runs its share of
+    // the items in turn; one tile per item (d = 256): one CTA per item
+    long long ctas = items;
+    if (NQ == 2) {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+            return FA_ERR_CUDA;
+        ctas = std::min<long long>(items, sms);
+    }
     dim3 grid(static_cast<unsigned>(ctas));
     ProfScope prof(0, stream);
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, pp);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -9,10 +9,12 @@
 // normalisation).  S and P live only in tensor memory ("FlashAttention原理概览"
 // section 3.1: the intermediate S_ij and P_ij never reach device memory).
 //
-// Decomposition (the outer-Q / inner-K/V order of 深度解析 section 四): one
-// CTA owns NQ query tiles of 128 rows of one (batch, head) and streams the
-// kept 128-key tiles of K and V through shared-memory rings of NSK (K) and
-// NSV (V) stages.  K gets the deeper ring: S of the next key tile is issued
+// Decomposition (the outer-Q / inner-K/V order of 深度解析 section 四): a
+// work item is NQ query tiles of 128 rows of one (batch, head); the kept
+// 128-key tiles of K and V stream through shared-memory rings of NSK (K) and
+// NSV (V) stages.  With NQ = 2 the grid is one CTA per SM and each CTA runs
+// its share of the items in turn (fwd_kernel describes the hand-over between
+// items); with NQ = 1 (d = 256) every item is its own CTA.  K gets the deeper ring: S of the next key tile is issued
 // right after P V of the current one, so its K tile is needed a whole
 // softmax phase before its V tile.
 //
@@ -24,9 +26,11 @@
 //                       writes P_t (16-bit) back over S_t and signals the MMA
 //                       warp once per half (keys 0..63, 64..127): O_t += P_t V
 //                       starts on the first half while the second is computed.
-//   warp 4*NQ           TMA producer: Q tiles once, then K_j per stage (and
-//                       V_j when NQ = 1).
-//   warp 4*NQ+2         (NQ = 2) TMA producer of the V_j tiles.
+//   warp 4*NQ           TMA producer: the item's Q tiles, then K_j per stage
+//                       (and V_j when NQ = 1).
+//   warp 4*NQ+2         (NQ = 2) TMA producer of the V_j tiles; it also issues
+//                       the TMA stores of each item's O (staged in V stages
+//                       0 .. NQ-1 by the softmax warps).
 //   warp 4*NQ+1         MMA issuer (one elected lane): S_t = Q_t K_j^T (SS form)
 //                       and O_t += P_t V_j (P read from TMEM, TS form).  It owns
 //                       the 512-column TMEM allocation.
@@ -55,6 +59,7 @@ struct FwdParams {
     int nqb;                  // query blocks of 128 rows
     int nkb;                  // key blocks of 128 keys
     int nbh;                  // batch x heads
+    int nitems;               // work items: nbh x ceil(nqb / NQ) query-tile groups
     int H;                    // heads (head of batch-head bh: bh % H)
     int mode;                 // kCausal (heaviest-first order) | kSparse bits
     float scale;
@@ -122,7 +127,12 @@ struct FwdCfg {
     static constexpr int kBarOFull = kBarPFull + NQ;
     static constexpr int kBarPFull2 = kBarOFull + NQ;   // P_t keys 64..127 in TMEM (kBarPFull: keys 0..63)
     static constexpr int kBarMmaDone = kBarPFull2 + NQ;
-    static constexpr int kNumBars = kBarMmaDone + 1;
+    // across work items (a CTA runs several in turn)
+    static constexpr int kBarQEmpty = kBarMmaDone + 1;  // every S product of the item has read Q
+    static constexpr int kBarOFree = kBarQEmpty + 1;    // [NQ] the epilogue has read O_t from TMEM
+    static constexpr int kBarOStaged = kBarOFree + NQ;  // O of every tile staged in shared memory
+    static constexpr int kBarStoreRead = kBarOStaged + 1;   // the TMA stores have read the staged O
+    static constexpr int kNumBars = kBarStoreRead + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;   // + slack for 1 KB alignment
     static constexpr int kSoftmaxWarps = 4 * NQ;
@@ -159,24 +169,50 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     }
 }
 
+// Work items: one per (batch-head, group of NQ query tiles), numbered query
+// group major and batch-head minor, so that under causal masking the heaviest
+// groups (the last query tiles) of every (b, h) come first.  A CTA runs the
+// items r * G + c (r even) and r * G + G - 1 - c (r odd) of the grid of G
+// CTAs, r = 0, 1, ...: heaviest first, and the back-and-forth order balances
+// the sums of a decreasing sequence (at B=4 H=16 N=4096 causal, 1,024 items on
+// 148 CTAs, the busiest CTA gets 1.02 x the mean work).
+__device__ __forceinline__ int fwd_item(int r, int c, int G) {
+    return r * G + ((r & 1) ? G - 1 - c : c);
+}
+
+template <int NQ>
+__device__ __forceinline__ void fwd_decode(const FwdParams &p, int item, int &bh, int &rb0) {
+    const int nqp = (p.nqb + NQ - 1) / NQ;
+    bh = item % p.nbh;
+    const int qi = item / p.nbh;
+    rb0 = ((p.mode & kCausal) ? nqp - 1 - qi : qi) * NQ;
+}
+
+// A CTA stays resident and runs its work items in turn.  Within an item the
+// roles work as described at the top of this file; across items:
+//   - the K producer loads the next item's Q once every S product of the
+//     current item has completed (QEmpty), so the first S of the next item
+//     follows the last P V of this one;
+//   - O_t is staged in V ring stage t (every P V of the item has completed
+//     when the epilogue runs) and written by TMA stores that the V producer
+//     issues before it loads the next item's V tiles (OStaged, StoreRead);
+//   - the MMA warp completes OFull_t of an item only after the epilogue of the
+//     item before has read O_t from TMEM (OFree_t), so each of these barriers
+//     completes once per item, in step with its waiter.
 template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, const FwdParams p) {
     using C = FwdCfg<D, NQ, NSK, NSV>;
+    static_assert(NSV >= NQ, "O_t is staged in V stage t");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // one-dimensional grid, (batch, head) minor: causal runs the heaviest
-    // query blocks of every (b, h) first (longest work first balances the SMs)
-    const int nqp = (p.nqb + NQ - 1) / NQ;
-    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
-    const int qi = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
-    const int qp = (p.mode & kCausal) ? nqp - 1 - qi : qi;
-    const int rb0 = qp * NQ;
+    const int cta = static_cast<int>(blockIdx.x);
+    const int G = static_cast<int>(gridDim.x);
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -197,8 +233,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             mbar_init(bar(C::kBarPFull + t), 128);
             mbar_init(bar(C::kBarPFull2 + t), 128);
             mbar_init(bar(C::kBarOFull + t), 1);
+            mbar_init(bar(C::kBarOFree + t), 128);
         }
         mbar_init(bar(C::kBarMmaDone), 1);
+        mbar_init(bar(C::kBarQEmpty), 1);
+        mbar_init(bar(C::kBarOStaged), 32 * C::kSoftmaxWarps);
+        mbar_init(bar(C::kBarStoreRead), 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -223,52 +263,94 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             // ------------------------------------------------------------ producer(s)
             const bool do_k = warp == C::kWarpTma;
             const bool do_v = warp == C::kWarpTmaV;
-            int nq_valid = 0;
-            for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
-            if (do_k && lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
-                for (int t = 0; t < NQ; ++t) {
-                    if (rb0 + t >= p.nqb) continue;
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
-                                    bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
-                }
-            }
-            __syncwarp();
-            KvIter<NQ, GENERAL> it;
-            int j;
-            uint32_t f;
-            int nk = 0, nv = 0;   // loads issued
-            bool ok = true;
-            while (ok && it.next(p, rb0, j, f)) {
-                if (do_k) {
-                    const int s = nk % NSK;
-                    ok = wait_bar(bar(C::kBarKEmpty + s), ((nk / NSK) & 1) ^ 1u, abort_flag);
-                    if (!ok) break;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
-                                        bar(C::kBarKFull + s), c * 64, j * 128, bh);
+            // TMA stores of item r's O tiles from V stages 0 .. NQ-1, once the
+            // softmax warps have staged them; the stages are reloaded only
+            // after the stores have read them
+            auto store_item = [&](int r, int bh, int rb0) -> bool {
+                const bool ok = wait_bar(bar(C::kBarOStaged), r & 1, abort_flag);
+                if (ok && lane == 0) {
+                    for (int t = 0; t < NQ; ++t) {
+                        if (rb0 + t >= p.nqb) continue;
+                        for (int c = 0; c < C::kChunks; ++c)   // rows >= Nq are clipped
+                            tma_store_3d(&tmo, sbase + C::kVOff + t * C::kTileBytes + c * C::kChunkBytes, c * 64,
+                                         (rb0 + t) * 128, bh);
                     }
-                    ++nk;
-                }
-                if (do_v) {
-                    const int s = nv % NSV;
-                    ok = wait_bar(bar(C::kBarVEmpty + s), ((nv / NSV) & 1) ^ 1u, abort_flag);
-                    if (!ok) break;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
-                                        bar(C::kBarVFull + s), c * 64, j * 128, bh);
-                    }
-                    ++nv;
+                    bulk_commit();
+                    bulk_wait_read();
+                    mbar_arrive(bar(C::kBarStoreRead));
                 }
                 __syncwarp();
+                return ok;
+            };
+            int nk = 0, nv = 0;   // loads issued (all items)
+            int nit = 0;          // items started
+            int pbh = 0, prb0 = 0;
+            bool ok = true;
+            for (int r = 0; ok; ++r) {
+                const int item = fwd_item(r, cta, G);
+                if (item >= p.nitems) break;
+                int bh, rb0;
+                fwd_decode<NQ>(p, item, bh, rb0);
+                if (do_v && r > 0) {
+                    ok = store_item(r - 1, pbh, prb0);
+                    if (!ok) break;
+                }
+                if (do_k) {
+                    if (r > 0) {
+                        ok = wait_bar(bar(C::kBarQEmpty), (r - 1) & 1, abort_flag);
+                        if (!ok) break;
+                    }
+                    if (lane == 0) {
+                        int nq_valid = 0;
+                        for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
+                        mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
+                        for (int t = 0; t < NQ; ++t) {
+                            if (rb0 + t >= p.nqb) continue;
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
+                                            bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
+                        }
+                    }
+                    __syncwarp();
+                }
+                ++nit;
+                KvIter<NQ, GENERAL> it;
+                int j;
+                uint32_t f;
+                while (ok && it.next(p, rb0, j, f)) {
+                    if (do_k) {
+                        const int s = nk % NSK;
+                        ok = wait_bar(bar(C::kBarKEmpty + s), ((nk / NSK) & 1) ^ 1u, abort_flag);
+                        if (!ok) break;
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
+                                            bar(C::kBarKFull + s), c * 64, j * 128, bh);
+                        }
+                        ++nk;
+                    }
+                    if (do_v) {
+                        const int s = nv % NSV;
+                        ok = wait_bar(bar(C::kBarVEmpty + s), ((nv / NSV) & 1) ^ 1u, abort_flag);
+                        if (!ok) break;
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
+                                            bar(C::kBarVFull + s), c * 64, j * 128, bh);
+                        }
+                        ++nv;
+                    }
+                    __syncwarp();
+                }
+                pbh = bh;
+                prb0 = rb0;
             }
+            // the last item's outputs
+            if (do_v && ok && nit > 0) store_item(nit - 1, pbh, prb0);
             // every issued load has landed before the CTA may exit
-            if (do_k) drain_bar(bar(C::kBarQ), 0);
+            if (do_k && nit > 0) drain_bar(bar(C::kBarQ), (nit - 1) & 1);
             for (int i = (nk > NSK ? nk - NSK : 0); i < nk; ++i)
                 drain_bar(bar(C::kBarKFull + i % NSK), (i / NSK) & 1);
             for (int i = (nv > NSV ? nv - NSV : 0); i < nv; ++i)
@@ -300,84 +382,113 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                            (acc || k > 0) ? 1u : 0u, leader);
             };
 
-            KvIter<NQ, GENERAL> it;
-            int j, jn;
-            uint32_t f, fn;
-            int cnt[NQ];
+            int kc = 0;        // K (= V) tiles consumed, all items
+            int pc[NQ];        // P_t V products issued, all items (parity of PFull_t)
 #pragma unroll
-            for (int t = 0; t < NQ; ++t) cnt[t] = 0;
-            bool have = it.next(p, rb0, j, f);
+            for (int t = 0; t < NQ; ++t) pc[t] = 0;
             bool ok = true;
-            if (have) {
-                ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag);
-                if (ok) {
+            for (int r = 0; ok; ++r) {
+                const int item = fwd_item(r, cta, G);
+                if (item >= p.nitems) break;
+                int bh, rb0;
+                fwd_decode<NQ>(p, item, bh, rb0);
+                (void)bh;
+                int ci[NQ];    // P_t V products of this item (accumulate after the first)
+#pragma unroll
+                for (int t = 0; t < NQ; ++t) ci[t] = 0;
+                KvIter<NQ, GENERAL> it;
+                int j, jn;
+                uint32_t f, fn;
+                bool have = it.next(p, rb0, j, f);
+                ok = wait_bar(bar(C::kBarQ), r & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (have) {
+                    const int s0 = kc % NSK;
+                    ok = wait_bar(bar(C::kBarKFull + s0), (kc / NSK) & 1, abort_flag);
+                    if (!ok) break;
                     tc_fence_after();
-                    {
-                        for (int t = 0; t < NQ; ++t)
-                            if ((f >> t) & 1u) {
-                                issue_s(t, 0);
-                                mma_commit(bar(C::kBarSFull + t), leader);
-                            }
-                        mma_commit(bar(C::kBarKEmpty), leader);
+                    for (int t = 0; t < NQ; ++t)
+                        if ((f >> t) & 1u) {
+                            issue_s(t, s0);
+                            mma_commit(bar(C::kBarSFull + t), leader);
+                        }
+                    mma_commit(bar(C::kBarKEmpty + s0), leader);
+                    __syncwarp();
+                } else {
+                    mma_commit(bar(C::kBarQEmpty), leader);   // no S product reads this Q
+                    __syncwarp();
+                }
+                int u = 0;
+                while (ok && have) {
+                    const int vi = kc + u;                 // V tile of this key tile
+                    const int s = vi % NSV;
+                    const uint32_t ph = (vi / NSV) & 1;
+                    const int ki = kc + u + 1;             // K tile of the next key tile
+                    const int sn = ki % NSK;
+                    const uint32_t phn = (ki / NSK) & 1;
+                    const bool have_n = it.next(p, rb0, jn, fn);
+                    if (!have_n) {
+                        // every S product of the item is issued: Q may be replaced
+                        mma_commit(bar(C::kBarQEmpty), leader);
+                        __syncwarp();
                     }
+                    ok = wait_bar(bar(C::kBarVFull + s), ph, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    bool k_ready = false;
+#pragma unroll
+                    for (int t = 0; t < NQ; ++t) {
+                        if ((f >> t) & 1u) {
+                            ok = wait_bar(bar(C::kBarPFull + t), pc[t] & 1, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(t, s, ci[t] > 0, 0, 4);
+                            __syncwarp();
+                            ok = wait_bar(bar(C::kBarPFull2 + t), pc[t] & 1, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(t, s, ci[t] > 0, 4, 8);
+                            __syncwarp();
+                            ++pc[t];
+                            ++ci[t];
+                        }
+                        if (have_n && ((fn >> t) & 1u)) {
+                            if (!k_ready) {
+                                ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_s(t, sn);
+                            mma_commit(bar(C::kBarSFull + t), leader);
+                            __syncwarp();
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(bar(C::kBarVEmpty + s), leader);
+                    if (have_n) mma_commit(bar(C::kBarKEmpty + sn), leader);
+                    __syncwarp();
+                    j = jn;
+                    f = fn;
+                    have = have_n;
+                    ++u;
+                }
+                if (!ok) break;
+                kc += u;
+                // O_t of this item is final once the products above complete;
+                // the item before must have read O_t first (one completion of
+                // OFull_t per item, in step with the epilogue that waits on it)
+                for (int t = 0; t < NQ; ++t) {
+                    if (r > 0) {
+                        ok = wait_bar(bar(C::kBarOFree + t), (r - 1) & 1, abort_flag);
+                        if (!ok) break;
+                    }
+                    mma_commit(bar(C::kBarOFull + t), leader);
                     __syncwarp();
                 }
             }
-            int u = 0;
-            while (ok && have) {
-                const int s = u % NSV;                 // V stage of this key tile
-                const uint32_t ph = (u / NSV) & 1;
-                const bool have_n = it.next(p, rb0, jn, fn);
-                const int sn = (u + 1) % NSK;          // K stage of the next key tile
-                const uint32_t phn = ((u + 1) / NSK) & 1;
-                ok = wait_bar(bar(C::kBarVFull + s), ph, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                bool k_ready = false;
-#pragma unroll
-                for (int t = 0; t < NQ; ++t) {
-                    if ((f >> t) & 1u) {
-                        ok = wait_bar(bar(C::kBarPFull + t), cnt[t] & 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(t, s, cnt[t] > 0, 0, 4);
-                        __syncwarp();
-                        ok = wait_bar(bar(C::kBarPFull2 + t), cnt[t] & 1, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(t, s, cnt[t] > 0, 4, 8);
-                        __syncwarp();
-                        ++cnt[t];
-                    }
-                    if (have_n && ((fn >> t) & 1u)) {
-                        if (!k_ready) {
-                            ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
-                            if (!ok) break;
-                            tc_fence_after();
-                            k_ready = true;
-                        }
-                        {
-                            issue_s(t, sn);
-                            mma_commit(bar(C::kBarSFull + t), leader);
-                        }
-                        __syncwarp();
-                    }
-                }
-                if (!ok) break;
-                {
-                    mma_commit(bar(C::kBarVEmpty + s), leader);
-                    if (have_n) mma_commit(bar(C::kBarKEmpty + sn), leader);
-                }
-                __syncwarp();
-                j = jn;
-                f = fn;
-                have = have_n;
-                ++u;
-            }
-            {
-                for (int t = 0; t < NQ; ++t) mma_commit(bar(C::kBarOFull + t), leader);
-                mma_commit(bar(C::kBarMmaDone), leader);
-            }
+            mma_commit(bar(C::kBarMmaDone), leader);
             __syncwarp();
             drain_bar(bar(C::kBarMmaDone), 0);
         }
@@ -386,200 +497,206 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int wq = warp & 3;
-        const int rb = rb0 + t;
         const int row_local = wq * 32 + lane;
-        const int row = rb * 128 + row_local;
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_off + 128u * t;
         const uint32_t tO = tmem + lane_off + C::kOCol + D * t;
         const float c = p.scale_log2;
-        float m = -INFINITY, l = 0.f, l_r = 0.f;
-        int cnt = 0;
-        // does this row see any key?  Taken from the band limits of the tiles
-        // it meets, not from m or l: a row that sees no key keeps m = -inf
-        // only while every masked score stays -inf, and the polynomial exp2
-        // gives masked scores 2^-125 instead of 0
-        bool seen = false;
-        KvIter<NQ, GENERAL> it;
-        int j;
-        uint32_t f;
+        int sc = 0;            // S_t products consumed, all items (parity of SFull_t)
         bool ok = true;
-        while (it.next(p, rb0, j, f)) {
-            if (!((f >> t) & 1u)) continue;
-            ok = wait_bar(bar(C::kBarSFull + t), cnt & 1, abort_flag);
+        for (int ri = 0; ok; ++ri) {
+            const int item = fwd_item(ri, cta, G);
+            if (item >= p.nitems) break;
+            int bh, rb0;
+            fwd_decode<NQ>(p, item, bh, rb0);
+            const int rb = rb0 + t;
+            const int row = rb * 128 + row_local;
+            float m = -INFINITY, l = 0.f, l_r = 0.f;
+            int cnt = 0;
+            // does this row see any key?  Taken from the band limits of the tiles
+            // it meets, not from m or l: a row that sees no key keeps m = -inf
+            // only while every masked score stays -inf, and the polynomial exp2
+            // gives masked scores 2^-125 instead of 0
+            bool seen = false;
+            KvIter<NQ, GENERAL> it;
+            int j;
+            uint32_t f;
+            while (it.next(p, rb0, j, f)) {
+                if (!((f >> t) & 1u)) continue;
+                ok = wait_bar(bar(C::kBarSFull + t), sc & 1, abort_flag);
+                if (!ok) break;
+                ++sc;
+                tc_fence_after();
+                uint32_t r[128];
+#pragma unroll
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
+                tmem_wait_ld(r);
+                // the scores as floats: a copy, not a float* view of r (reading
+                // the asm-written integers through another type is undefined and
+                // let stale register values into the row max)
+                float sv[128];
+#pragma unroll
+                for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
+                // this row's visible keys within the tile: [lo, hi]
+                int lo, hi, rk = 0;
+                if constexpr (GENERAL) {
+                    rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
+                    lo = max(rk - p.wl, -1);
+                    hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
+                } else {
+                    lo = -1;
+                    hi = 127;
+                    if ((p.mode & kCausal) && j == rb) hi = row_local;                    // diagonal tile
+                    if (j == p.nkb - 1 && (p.Nk & 127)) hi = min(hi, (p.Nk & 127) - 1);  // key tail
+                }
+                seen |= max(lo, 0) <= min(hi, 127);
+                if (GENERAL && p.alibi) {
+                    // score + bias / scale, bias = -slope |row + off - key|
+                    const float sl = -p.alibi[bh % p.H] / p.scale;
+                    const float base = static_cast<float>(rk);
+#pragma unroll
+                    for (int k = 0; k < 128; ++k) sv[k] = fmaf(sl, fabsf(base - static_cast<float>(k)), sv[k]);
+                }
+                if (__any_sync(0xffffffffu, lo > 0 || hi < 127)) {
+#pragma unroll
+                    for (int k = 0; k < 128; ++k)
+                        if (k < lo || k > hi) sv[k] = -INFINITY;
+                }
+                // row max: four independent chains of three-input max
+                float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+                for (int k = 4; k < 128; k += 8) {
+                    mx0 = fmax3(mx0, sv[k], sv[k + 1]);
+                    mx1 = fmax3(mx1, sv[k + 2], sv[k + 3]);
+                    mx2 = fmax3(mx2, sv[k + 4], sv[k + 5]);
+                    mx3 = fmax3(mx3, sv[k + 6], sv[k + 7]);
+                }
+                const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+                const float m_cand = fmaxf(m, mx * c);
+                const bool grow = m_cand > m + 8.0f;    // lazy: keep m unless it moves by > 2^8
+                const float m_new = grow ? m_cand : m;
+                const float alpha = grow ? ex2(m - m_new) : 1.0f;
+                const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
+                if (cnt > 0 && __any_sync(0xffffffffu, grow)) {
+                    // S_t's completion implies the previous O_t += P V finished
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32_wait(tO + 32 * q, o);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st32(tO + 32 * q, o);
+                    }
+                }
+                // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA
+                // pipe (polynomial) instead of the special-function unit.  Measured
+                // on B200: at d = 128 and 256 moving any pairs made the softmax
+                // slower (issue-bound); at d = 64 two of eight were 4.7 % faster
+                // but failed the parity of a causal cross-attention case (Nq = 300,
+                // Nk = 100) not yet explained, so every pair uses the special-
+                // function unit.
+                constexpr int kPolyPairs = 0;
+                float2 acc[4], acc_r[4];
+#pragma unroll
+                for (int a4 = 0; a4 < 4; ++a4) acc[a4] = acc_r[a4] = make_float2(0.f, 0.f);
+                const float2 cc = make_float2(c, c), mm = make_float2(-m_use, -m_use);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int g = 16 * q + k;
+                        const float2 x = ffma2(make_float2(sv[2 * g], sv[2 * g + 1]), cc, mm);
+                        float2 pr;
+                        if ((g & 7) >= 8 - kPolyPairs) {
+                            pr = exp2_poly2(x);
+                        } else {
+                            pr.x = ex2(x.x);
+                            pr.y = ex2(x.y);
+                        }
+                        pk[k] = pack2<BF16>(pr.x, pr.y);
+                        acc[k & 3] = fadd2(acc[k & 3], pr);
+                        if constexpr (BF16) {
+                            // O is normalised by the sum of the same rounded P the
+                            // tensor core multiplies (a row dominated by one key then
+                            // comes out exact); LSE keeps the unrounded sum
+                            acc_r[k & 3] = fadd2(acc_r[k & 3], unpack2<true>(pk[k]));
+                        }
+                    }
+                    tmem_st16(tS + 16 * q, pk);
+                    if (q == 1) {
+                        // the first 64 keys of P_t are in TMEM: the MMA warp can start
+                        // O_t += P_t V on them while the second half is computed
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(bar(C::kBarPFull + t));
+                    }
+                }
+                const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+                const float sum = s01.x + s01.y;
+                float sum_r = 0.f;
+                if constexpr (BF16) {
+                    const float2 r01 = fadd2(fadd2(acc_r[0], acc_r[1]), fadd2(acc_r[2], acc_r[3]));
+                    sum_r = r01.x + r01.y;
+                }
+                l = l * alpha + sum;
+                if constexpr (BF16) l_r = l_r * alpha + sum_r;
+                m = m_new;
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull2 + t));
+                ++cnt;
+            }
+            if (!ok) break;
+            // ---------------------------------------------------------- epilogue
+            ok = wait_bar(bar(C::kBarOFull + t), ri & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[128];
-#pragma unroll
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
-            tmem_wait_ld(r);
-            // the scores as floats: a copy, not a float* view of r (reading
-            // the asm-written integers through another type is undefined and
-            // let stale register values into the row max)
-            float sv[128];
-#pragma unroll
-            for (int k = 0; k < 128; ++k) sv[k] = __uint_as_float(r[k]);
-            // this row's visible keys within the tile: [lo, hi]
-            int lo, hi, rk = 0;
-            if constexpr (GENERAL) {
-                rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
-                lo = max(rk - p.wl, -1);
-                hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
-            } else {
-                lo = -1;
-                hi = 127;
-                if ((p.mode & kCausal) && j == rb) hi = row_local;                    // diagonal tile
-                if (j == p.nkb - 1 && (p.Nk & 127)) hi = min(hi, (p.Nk & 127) - 1);  // key tail
+            // O_t is staged in V stage t (every P V of the item has completed)
+            // once the previous item's stores have read it, as 128-byte-swizzled
+            // 64-column chunks for the V producer's TMA stores
+            if (ri > 0) {
+                ok = wait_bar(bar(C::kBarStoreRead), (ri - 1) & 1, abort_flag);
+                if (!ok) break;
             }
-            seen |= max(lo, 0) <= min(hi, 127);
-            if (GENERAL && p.alibi) {
-                // score + bias / scale, bias = -slope |row + off - key|
-                const float sl = -p.alibi[bh % p.H] / p.scale;
-                const float base = static_cast<float>(rk);
-#pragma unroll
-                for (int k = 0; k < 128; ++k) sv[k] = fmaf(sl, fabsf(base - static_cast<float>(k)), sv[k]);
-            }
-            if (__any_sync(0xffffffffu, lo > 0 || hi < 127)) {
-#pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    if (k < lo || k > hi) sv[k] = -INFINITY;
-            }
-            // row max: four independent chains of three-input max
-            float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
-#pragma unroll
-            for (int k = 4; k < 128; k += 8) {
-                mx0 = fmax3(mx0, sv[k], sv[k + 1]);
-                mx1 = fmax3(mx1, sv[k + 2], sv[k + 3]);
-                mx2 = fmax3(mx2, sv[k + 4], sv[k + 5]);
-                mx3 = fmax3(mx3, sv[k + 6], sv[k + 7]);
-            }
-            const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
-            const float m_cand = fmaxf(m, mx * c);
-            const bool grow = m_cand > m + 8.0f;    // lazy: keep m unless it moves by > 2^8
-            const float m_new = grow ? m_cand : m;
-            const float alpha = grow ? ex2(m - m_new) : 1.0f;
-            const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-            if (cnt > 0 && __any_sync(0xffffffffu, grow)) {
-                // S_t's completion implies the previous O_t += P V finished
+            if (rb < p.nqb) {
+                uint8_t *stage = smem + C::kVOff + t * C::kTileBytes;
+                const float l_o = BF16 ? l_r : l;
+                // a row that saw no key: O = 0, LSE = -inf
+                const float inv_l = (seen && l_o > 0.f) ? 1.0f / l_o : 0.0f;
 #pragma unroll 1
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t o[32];
-                    tmem_ld32_wait(tO + 32 * q, o);
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                    tmem_st32(tO + 32 * q, o);
-                }
-            }
-            // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA
-            // pipe (polynomial) instead of the special-function unit.  Measured
-            // on B200: at d = 128 and 256 moving any pairs made the softmax
-            // slower (issue-bound); at d = 64 two of eight were 4.7 % faster
-            // but failed the parity of a causal cross-attention case (Nq = 300,
-            // Nk = 100) not yet explained, so every pair uses the special-
-            // function unit.
-            constexpr int kPolyPairs = 0;
-            float2 acc[4], acc_r[4];
-#pragma unroll
-            for (int a4 = 0; a4 < 4; ++a4) acc[a4] = acc_r[a4] = make_float2(0.f, 0.f);
-            const float2 cc = make_float2(c, c), mm = make_float2(-m_use, -m_use);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int g = 16 * q + k;
-                    const float2 x = ffma2(make_float2(sv[2 * g], sv[2 * g + 1]), cc, mm);
-                    float2 pr;
-                    if ((g & 7) >= 8 - kPolyPairs) {
-                        pr = exp2_poly2(x);
+                    if (cnt > 0) {
+                        tmem_ld32_wait(tO + 32 * q, o);
                     } else {
-                        pr.x = ex2(x.x);
-                        pr.y = ex2(x.y);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = 0u;
                     }
-                    pk[k] = pack2<BF16>(pr.x, pr.y);
-                    acc[k & 3] = fadd2(acc[k & 3], pr);
-                    if constexpr (BF16) {
-                        // O is normalised by the sum of the same rounded P the
-                        // tensor core multiplies (a row dominated by one key then
-                        // comes out exact); LSE keeps the unrounded sum
-                        acc_r[k & 3] = fadd2(acc_r[k & 3], unpack2<true>(pk[k]));
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        pk[k] = pack2<BF16>(__uint_as_float(o[2 * k]) * inv_l,
+                                            __uint_as_float(o[2 * k + 1]) * inv_l);
+                    uint8_t *srow = stage + (q >> 1) * C::kChunkBytes + row_local * 128;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int u = (q & 1) * 4 + k;   // 16-byte unit within the 128-byte row
+                        *reinterpret_cast<uint4 *>(srow + ((u ^ (row_local & 7)) << 4)) =
+                            make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                     }
                 }
-                tmem_st16(tS + 16 * q, pk);
-                if (q == 1) {
-                    // the first 64 keys of P_t are in TMEM: the MMA warp can start
-                    // O_t += P_t V on them while the second half is computed
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(bar(C::kBarPFull + t));
+                if (row < p.Nq) {
+                    const float lse = (seen && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                    p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
                 }
             }
-            const float2 s01 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-            const float sum = s01.x + s01.y;
-            float sum_r = 0.f;
-            if constexpr (BF16) {
-                const float2 r01 = fadd2(fadd2(acc_r[0], acc_r[1]), fadd2(acc_r[2], acc_r[3]));
-                sum_r = r01.x + r01.y;
-            }
-            l = l * alpha + sum;
-            if constexpr (BF16) l_r = l_r * alpha + sum_r;
-            m = m_new;
-            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull2 + t));
-            ++cnt;
-        }
-        if (ok && cnt > 0) ok = wait_bar(bar(C::kBarOFull + t), 0, abort_flag);
-        tc_fence_after();
-        // O_t is staged in the Q_t buffer (every S product has completed once
-        // O_t is final) as 128-byte-swizzled 64-column chunks, then written by
-        // TMA stores: one thread per row would touch 32 lines per store
-        const bool epi = rb < p.nqb && ok;
-        uint8_t *stage = smem + C::kQOff + t * C::kTileBytes;
-        // a tile that saw no key block never waited for its Q load: it must
-        // land before the staging area is written
-        if (epi && cnt == 0) drain_bar(bar(C::kBarQ), 0);
-        if (epi) {
-            const bool valid = row < p.Nq;
-            const float l_o = BF16 ? l_r : l;
-            // a row that saw no key: O = 0, LSE = -inf
-            const float inv_l = (seen && l_o > 0.f) ? 1.0f / l_o : 0.0f;
-#pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t o[32];
-                if (cnt > 0) {
-                    tmem_ld32_wait(tO + 32 * q, o);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = 0u;
-                }
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    pk[k] = pack2<BF16>(__uint_as_float(o[2 * k]) * inv_l,
-                                        __uint_as_float(o[2 * k + 1]) * inv_l);
-                uint8_t *srow = stage + (q >> 1) * C::kChunkBytes + row_local * 128;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int u = (q & 1) * 4 + k;   // 16-byte unit within the 128-byte row
-                    *reinterpret_cast<uint4 *>(srow + ((u ^ (row_local & 7)) << 4)) =
-                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-                }
-            }
-            if (valid) {
-                const float lse = (seen && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
-            }
-        }
-        fence_async_smem();
-        named_sync(1 + t, 128);   // the four warps of query tile t (every one of them gets here)
-        if (epi && wq == 0 && lane == 0) {
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_store_3d(&tmo, smem_u32(stage + c * C::kChunkBytes), c * 64, rb * 128, bh);   // rows >= Nq clipped
-            bulk_commit();
-            bulk_wait_read();   // shared memory stays allocated until the stores have read it
+            mbar_arrive(bar(C::kBarOFree + t));     // O_t read: the next item may complete OFull_t
+            fence_async_smem();
+            mbar_arrive(bar(C::kBarOStaged));      // staged O visible to the TMA stores
         }
     }
 
