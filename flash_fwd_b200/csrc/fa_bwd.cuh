@@ -203,18 +203,28 @@ struct BwdCfg {
     static constexpr int kdSOff = kdOOff + NS * kQTile;   // dS^T: [2 query chunks][128 keys][64 queries]
     static constexpr int kStatBytes = BM * 4;
     static constexpr int kStatOff = kdSOff + 2 * kChunk;  // per stage: LSE log2 e [BM], D [BM]
-    static constexpr int kBarOff = kStatOff + NS * 2 * kStatBytes;
+    // d = 64: dQ of a query tile is staged as two halves [64 queries][64 d]
+    // fp32 and added to the accumulator with bulk reductions (whole-line
+    // requests; the per-lane reductions of an M = 64 product are 64 bytes)
+    static constexpr int kDqHalf = 64 * D * 4;
+    static constexpr int kDqStageOff = kStatOff + NS * 2 * kStatBytes;
+    static constexpr int kDqStageBytes = D == 64 ? 2 * kDqHalf : 0;
+    static constexpr int kBarOff = kDqStageOff + kDqStageBytes;
     static constexpr int kBarKV = 0;
-    static constexpr int kBarQFull = 1;
+    static constexpr int kBarQFull = 1;                   // Q_i and LSE_i landed
     static constexpr int kBarQEmpty = kBarQFull + NS;
-    static constexpr int kBarSFull = kBarQEmpty + NS;     // S^T computed
+    static constexpr int kBarOFull = kBarQEmpty + NS;     // dO_i and D_i landed
+    static constexpr int kBarOEmpty = kBarOFull + NS;
+    static constexpr int kBarSFull = kBarOEmpty + NS;     // S^T computed
     static constexpr int kBarDPFull = kBarSFull + 1;      // dP^T computed
     static constexpr int kBarPFull = kBarDPFull + 1;      // P^T in TMEM (256 arrivals)
     static constexpr int kBarDsFull = kBarPFull + 1;      // dS^T in smem, dP^T read (256 arrivals)
     static constexpr int kBarDqFull = kBarDsFull + 1;     // dQ^T computed
     static constexpr int kBarDqFree = kBarDqFull + 1;     // dQ^T read out (128 arrivals)
     static constexpr int kBarMmaDone = kBarDqFree + 1;
-    static constexpr int kNumBars = kBarMmaDone + 1;
+    static constexpr int kBarDqStageFree = kBarMmaDone + 1;   // d = 64: staging half free (issuing thread)
+    static constexpr int kBarDqStaged = kBarDqStageFree + 1;  // d = 64: staging half written (128 arrivals)
+    static constexpr int kNumBars = kBarDqStaged + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // No alignment slack: the kernel checks that dynamic shared memory starts
     // on a 1 KB boundary (the 128-byte swizzle atoms need it).
@@ -229,6 +239,9 @@ struct BwdCfg {
     static constexpr int kColDP = 128;
     static constexpr int kColDV = 256;
     static constexpr int kColDK = 256 + D;
+    // dQ^T: its own columns at d = 64 (free there), so dP^T of the next tile
+    // need not wait for the drain; at d = 128 it reuses the dP^T columns
+    static constexpr int kColDQ = D == 64 ? 384 : kColDP;
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -266,6 +279,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(bar(C::kBarQFull + s), 1);
             mbar_init(bar(C::kBarQEmpty + s), 1);
+            mbar_init(bar(C::kBarOFull + s), 1);
+            mbar_init(bar(C::kBarOEmpty + s), 1);   // dP^T(i) and dV(i) have read dO_i
         }
         mbar_init(bar(C::kBarSFull), 1);
         mbar_init(bar(C::kBarDPFull), 1);
@@ -274,6 +289,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bar(C::kBarDqFull), 1);
         mbar_init(bar(C::kBarDqFree), 128);
         mbar_init(bar(C::kBarMmaDone), 1);
+        mbar_init(bar(C::kBarDqStageFree), 1);
+        mbar_init(bar(C::kBarDqStaged), 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -310,27 +327,38 @@ __global__ void __launch_bounds__(512, 1)
             int i;
             while (it.next(p, j, i)) {
                 const int s = cnt % NS;
+                // Q_i with the padded LSE_i, dO_i with D_i (TMA tiles and bulk
+                // copies of the statistics prepared by bwd_pre), each pair on
+                // its own transaction barrier
+                const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
+                const uint32_t st = sbase + C::kStatOff + s * 2 * C::kStatBytes;
                 ok = wait_bar(bar(C::kBarQEmpty + s), ((cnt / NS) & 1) ^ 1u, abort_flag);
                 if (!ok) break;
-                // Q_i, dO_i (TMA tiles) and the padded per-row statistics (bulk
-                // copies, prepared by bwd_pre) land on one transaction barrier
                 if (lane == 0) {
                     const uint32_t qb = bar(C::kBarQFull + s);
-                    mbar_arrive_expect_tx(qb, 2 * C::kQTile + 2 * C::kStatBytes);
-                    for (int c = 0; c < D / 64; ++c) {
+                    mbar_arrive_expect_tx(qb, C::kQTile + C::kStatBytes);
+                    for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kChunk, &tmq, qb, c * 64, i * BM, bh);
-                        tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kChunk, &tmdo, qb, c * 64, i * BM, bh);
-                    }
-                    const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
-                    const uint32_t st = sbase + C::kStatOff + s * 2 * C::kStatBytes;
                     bulk_load(st, p.lse2 + srow, C::kStatBytes, qb);
-                    bulk_load(st + C::kStatBytes, p.dvec + srow, C::kStatBytes, qb);
+                }
+                __syncwarp();
+                ok = wait_bar(bar(C::kBarOEmpty + s), ((cnt / NS) & 1) ^ 1u, abort_flag);
+                if (!ok) break;
+                if (lane == 0) {
+                    const uint32_t ob = bar(C::kBarOFull + s);
+                    mbar_arrive_expect_tx(ob, C::kQTile + C::kStatBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kChunk, &tmdo, ob, c * 64, i * BM, bh);
+                    bulk_load(st + C::kStatBytes, p.dvec + srow, C::kStatBytes, ob);
                 }
                 __syncwarp();
                 ++cnt;
             }
             drain_bar(bar(C::kBarKV), 0);
-            for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
+            for (int x = (cnt > NS ? cnt - NS : 0); x < cnt; ++x) {
+                drain_bar(bar(C::kBarQFull + x % NS), (x / NS) & 1);
+                drain_bar(bar(C::kBarOFull + x % NS), (x / NS) & 1);
+            }
         } else if (warp == C::kWarpMma) {
             // ------------------------------------------------------------ MMA issuer
             const uint32_t leader = elect_one();   // the lane that issues tcgen05 ops
@@ -376,7 +404,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (with_dq) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k)      // dQ^T (D x BM) = K_j^T dS^T, over the 128 keys
-                        mma_ss(tmem + C::kColDP, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u,
+                        mma_ss(tmem + C::kColDQ, dK_mn.at(k * 2048), ddS_mn.at(k * 2048), kIdQ, k > 0 ? 1u : 0u,
                                leader);
                 }
             };
@@ -388,12 +416,15 @@ __global__ void __launch_bounds__(512, 1)
                 ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
                 if (ok) {
                     tc_fence_after();
-                    {
-                        issue_s(0);
-                        mma_commit(bar(C::kBarSFull), leader);
-                        issue_dp(0);
-                        mma_commit(bar(C::kBarDPFull), leader);
-                    }
+                    issue_s(0);
+                    mma_commit(bar(C::kBarSFull), leader);
+                    __syncwarp();
+                    ok = wait_bar(bar(C::kBarOFull), 0, abort_flag);
+                }
+                if (ok) {
+                    tc_fence_after();
+                    issue_dp(0);
+                    mma_commit(bar(C::kBarDPFull), leader);
                     __syncwarp();
                 }
             }
@@ -406,6 +437,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (!ok) break;
                 tc_fence_after();
                 issue_dv(s, cnt > 0);
+                mma_commit(bar(C::kBarOEmpty + s), leader);   // dP^T(i), dV(i): the readers of dO_i
                 __syncwarp();
                 if (have_n) {
                     ok = wait_bar(bar(C::kBarQFull + sn), ((cnt + 1) / NS) & 1, abort_flag);
@@ -419,6 +451,11 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 ok = wait_bar(bar(C::kBarDsFull), ph, abort_flag);
                 if (!ok) break;
+                if (D == 64 && with_dq && cnt > 0) {
+                    // dQ^T has its own columns: the drain must have read out the previous tile's
+                    ok = wait_bar(bar(C::kBarDqFree), (cnt - 1) & 1, abort_flag);
+                    if (!ok) break;
+                }
                 tc_fence_after();
                 {
                     issue_dk_dq(s, cnt > 0);
@@ -427,8 +464,12 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 __syncwarp();
                 if (have_n) {
-                    // without dQ^T the dP^T columns are free once dS(i) is in place
-                    ok = !with_dq || wait_bar(bar(C::kBarDqFree), ph, abort_flag);
+                    // the dP^T columns are free once dS(i) is in place, unless
+                    // dQ^T(i) was written over them (d = 128): then once the
+                    // drain has read it out
+                    ok = !with_dq || D == 64 || wait_bar(bar(C::kBarDqFree), ph, abort_flag);
+                    if (!ok) break;
+                    ok = wait_bar(bar(C::kBarOFull + sn), ((cnt + 1) / NS) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     {
@@ -527,7 +568,8 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarPFull));
                 // phase B: dS^T = P^T o (dP^T - D), with the 16-bit P^T
-                ok = wait_bar(bar(C::kBarDPFull), ph, abort_flag);
+                ok = wait_bar(bar(C::kBarDPFull), ph, abort_flag) &&
+                     wait_bar(bar(C::kBarOFull + s), (cnt / NS) & 1, abort_flag);   // D_i
                 if (!ok) break;
                 tc_fence_after();
                 {
@@ -615,6 +657,8 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
             const bool row_lane = (D == 128) || (lane < 16);
             const int dcol = (D == 128) ? wq * 32 + lane : wq * 16 + (lane & 15);
+            const bool issuer = wq == 0 && lane == 0;   // d = 64: issues the bulk reductions
+            int nh = 0;                                  // d = 64: staged halves
             QIter<BM, GENERAL> it;
             int i;
             while (p.dqacc != nullptr && it.next(p, j, i)) {
@@ -623,15 +667,53 @@ __global__ void __launch_bounds__(512, 1)
                 tc_fence_after();
                 uint32_t v[BM];
                 // 128 registers: four loads and one wait (a single load-and-wait
-                // statement does not fit this kernel's register budget); v is
-                // only read after the wait
+                // statement does not fit this kernel's register budget); the
+                // wait names every loaded register
 #pragma unroll
                 for (int ch = 0; ch < BM / 32; ++ch)
-                    tmem_ld32(tmem + lane_off + C::kColDP + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
+                    tmem_ld32(tmem + lane_off + C::kColDQ + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * ch]));
                 tmem_wait_ld(v);
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarDqFree));
-                if (row_lane) {
+                if constexpr (D == 64) {
+                    // two halves of 64 queries: [64 queries][64 d] fp32 in the
+                    // staging half h, then one bulk reduction of the contiguous
+                    // rows into the accumulator (unrolled: v is indexed by h).
+                    // The four drain warps hand over through mbarriers with
+                    // bounded waits, so that none can be left waiting.
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int q0 = i * BM + 64 * h;
+                        const int rows = min(64, p.Nq - q0);
+                        if (rows <= 0) break;
+                        // staging half h was last read by the reduction two before
+                        if (issuer) {
+                            bulk_wait_read_1();
+                            mbar_arrive(bar(C::kBarDqStageFree));
+                        }
+                        ok = wait_bar(bar(C::kBarDqStageFree), nh & 1, abort_flag);
+                        if (!ok) break;
+                        if (row_lane) {
+                            float *st = reinterpret_cast<float *>(smem + C::kDqStageOff + h * C::kDqHalf) + dcol;
+#pragma unroll
+                            for (int k = 0; k < 64; ++k) st[k * D] = __uint_as_float(v[64 * h + k]);
+                        }
+                        fence_async_smem();
+                        mbar_arrive(bar(C::kBarDqStaged));
+                        if (wq == 0) {
+                            ok = wait_bar(bar(C::kBarDqStaged), nh & 1, abort_flag);
+                            if (!ok) break;
+                            if (issuer) {
+                                bulk_reduce_add_f32(p.dqacc + (static_cast<size_t>(bh) * p.Nq + q0) * D,
+                                                    sbase + C::kDqStageOff + h * C::kDqHalf,
+                                                    static_cast<uint32_t>(rows) * D * 4);
+                                bulk_commit();
+                            }
+                        }
+                        ++nh;
+                    }
+                    if (!ok) break;
+                } else if (row_lane) {
                     float *acc = p.dqacc + (static_cast<size_t>(bh) * p.Nq + static_cast<size_t>(i) * BM) * D + dcol;
                     const int lim = p.Nq - i * BM;
 #pragma unroll
@@ -640,6 +722,8 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 ++cnt;
             }
+            // the staged dQ must be read, and added, before the CTA exits
+            if (D == 64 && issuer) bulk_wait_all();
         }
     }
 

@@ -157,7 +157,20 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
                  "r"(src), "r"(x), "r"(y), "r"(z)
                  : "memory");
 }
+// global[dst .. dst + bytes) += shared[src ..] in fp32, element by element,
+// as one bulk reduction (both addresses 16-byte aligned, bytes % 16 == 0);
+// tracked by this thread's bulk groups like the TMA stores.
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(dst)),
+                 "r"(src), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most one committed bulk group has not finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// Waits until every committed bulk group has completed (its global writes included).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Waits until the committed bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Makes this thread's generic-proxy shared-memory writes visible to TMA.
@@ -447,6 +460,12 @@ struct SmemDesc {
 };
 __device__ __forceinline__ SmemDesc make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     const uint64_t d = smem_desc_sw128(saddr, lbo, sbo);
+    return SmemDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+// The same for a 64-byte-swizzled operand (rows of 64 bytes, 8-row atoms of
+// 512 bytes: sbo = 512; swizzle mode 4 at [61,64)).
+__device__ __forceinline__ SmemDesc make_desc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    const uint64_t d = (smem_desc_sw128(saddr, lbo, sbo) & ~(7ull << 61)) | (4ull << 61);
     return SmemDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
 }
 
