@@ -62,6 +62,8 @@ WORKLOADS = {
     # the FP8 forward (block quantisation + incoherent processing) on the same shape:
     # a step quantises the bf16 Q, K, V and runs the E4M3 forward
     "fp8_128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
+    "fp8_64": dict(B=4, H=16, N=4096, d=64, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
+    "fp8_256": dict(B=4, H=16, N=4096, d=256, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
 }
 
 

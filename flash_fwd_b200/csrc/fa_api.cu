@@ -95,11 +95,13 @@ int make_map8(CUtensorMap *map, const void *base, int d, int N, long long BH) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
                              static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(d), 128, 1};
+    // one swizzle atom wide: 128 bytes (d = 256: two boxes per 128-row
+    // tile), or 64 bytes with the 64-byte swizzle at d = 64
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(d < 128 ? d : 128), 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, d < 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -416,6 +418,20 @@ int launch_quant(const fa::QuantParams &qp, long long BH, cudaStream_t s) {
     return FA_OK;
 }
 
+// The FP8 forward: one CTA per NQ query tiles of one (b, h), heaviest first under causal.
+template <int D, bool BF16>
+int launch_fwd8(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mo,
+                const fa::Fwd8Params &p, long long BH, cudaStream_t s) {
+    using C = fa::Fwd8Cfg<D>;
+    auto kern = fa::fwd8_kernel<D, BF16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(BH * ((p.nb + C::NQ - 1) / C::NQ)));
+    ProfScope prof(6, s);
+    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -465,9 +481,9 @@ FA_API int fa_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, c
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (out_dtype != FA_F16 && out_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     const long long BH = static_cast<long long>(B) * H;
-    if (N > fa::kMaxRows || BH * ((N + 255) / 256) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    if (N > fa::kMaxRows || BH * ((N + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     const void *ptrs[] = {q8, k8, v8, o, lse};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
@@ -490,15 +506,15 @@ FA_API int fa_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, c
     p.nbh = static_cast<int>(BH);
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * kLog2e;
-    using C = fa::Fwd8Cfg;
-    auto kern = out_dtype == FA_BF16 ? fa::fwd8_kernel<true> : fa::fwd8_kernel<false>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-        return FA_ERR_CUDA;
-    const dim3 grid(static_cast<unsigned>(BH * ((p.nb + 1) / 2)));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    ProfScope prof(6, s);
-    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(mq, mk, mv, mo, p);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if (d == 64)
+        return out_dtype == FA_BF16 ? launch_fwd8<64, true>(mq, mk, mv, mo, p, BH, s)
+                                    : launch_fwd8<64, false>(mq, mk, mv, mo, p, BH, s);
+    if (d == 128)
+        return out_dtype == FA_BF16 ? launch_fwd8<128, true>(mq, mk, mv, mo, p, BH, s)
+                                    : launch_fwd8<128, false>(mq, mk, mv, mo, p, BH, s);
+    return out_dtype == FA_BF16 ? launch_fwd8<256, true>(mq, mk, mv, mo, p, BH, s)
+                                : launch_fwd8<256, false>(mq, mk, mv, mo, p, BH, s);
 }
 
 FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,

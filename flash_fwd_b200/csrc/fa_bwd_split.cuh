@@ -50,6 +50,13 @@ struct BwdSplitCfg {
     static constexpr int kDqCols = DQT ? BM : DH;         // fp32 columns per drain thread
     static constexpr int kColPT = DQT ? 192 : 448;        // NPB buffers of 16-bit P^T (BM / 2 columns each)
     static constexpr int kStatBytes = BM * 4;
+    // CTA order: heads in groups of kHeadGroup, key-block columns major within
+    // a group (heaviest first under causal), heads minor; the running CTAs then
+    // reduce into the fp32 dQ rows of kHeadGroup heads only (at d = 256 the
+    // accumulator of all heads is far larger than L2).  Measured at B=4 H=16
+    // N=4096 causal: 3.99 ms per launch with one group of all 64 heads, 3.70
+    // with groups of 4 or 8, 3.75 with 16
+    static constexpr int kHeadGroup = 8;
     static_assert(kColPT + NPB * BM / 2 <= (DQT ? 256 : 512), "P^T columns");
     static_assert(DQT ? (BM == 64 && DH == 128) : (BM == 128 && DH == 64), "tile shape");
     static_assert(kColDQ + kDqCols <= 512 && kColDK + DH <= 512, "TMEM columns");
@@ -71,9 +78,18 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // one-dimensional grid, (batch, head) minor (see bwd_kernel)
-    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
-    const int jh = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    // one-dimensional grid: groups of kHeadGroup heads, (batch, head) minor
+    // within a group (see bwd_kernel)
+    int bh, jh;
+    {
+        const int hg = min(C::kHeadGroup, p.nbh);
+        const long long per = static_cast<long long>(hg) * p.nkb * DSPLIT;
+        const int g = static_cast<int>(blockIdx.x / per);
+        const int r = static_cast<int>(blockIdx.x - g * per);
+        const int gh = min(hg, p.nbh - g * hg);   // heads in this group
+        jh = r / gh;
+        bh = g * hg + (r - jh * gh);
+    }
     const int j = jh / DSPLIT;
     const int h = jh % DSPLIT;
 

@@ -28,12 +28,14 @@
 //                      consecutive channels; butterflies below d/32 run in the
 //                      lane, the others across lanes with shuffles.
 //   fp8_vscale_kernel  the head's V scale, written to every block slot.
-//   fwd8_kernel        the forward of fa_fwd.cuh (d = 128, two 128-row query
-//                      tiles per CTA, dense or causal) on E4M3 operands:
-//                      Q8, K8, V8 tiles are 16 KB (one 128-byte swizzle atom
-//                      wide), P8 takes 32 TMEM columns (four codes per column)
-//                      over S, O tiles are staged in the finished K ring and
-//                      written by TMA stores.
+//   fwd8_kernel        the forward of fa_fwd.cuh (dense or causal) on E4M3
+//                      operands: d = 64 and 128 with two 128-row query tiles
+//                      per CTA, d = 256 with one (its O accumulator takes 256
+//                      TMEM columns).  Q8, K8, V8 tiles are swizzle atoms of
+//                      128-byte rows (two per tile at d = 256; 64-byte rows
+//                      with the 64-byte swizzle at d = 64), P8 takes 32 TMEM
+//                      columns (four codes per column) over S, O tiles are
+//                      staged in the finished K ring and written by TMA stores.
 #pragma once
 
 #include "fa_fwd.cuh"
@@ -199,7 +201,7 @@ __global__ void fp8_vscale_kernel(float *sv, int nb, long long BH) {
 }
 
 // ---------------------------------------------------------------------------
-// FP8 forward (d = 128)
+// FP8 forward (d = 64, 128, 256)
 // ---------------------------------------------------------------------------
 struct Fwd8Params {
     float *lse;               // [BH][N]
@@ -210,10 +212,17 @@ struct Fwd8Params {
     float scale_log2;         // scale * log2(e)
 };
 
+template <int D>
 struct Fwd8Cfg {
-    static constexpr int D = 128;
-    static constexpr int NQ = 2, NSK = 6, NSV = 4;
-    static constexpr int kTileBytes = 128 * D;          // 128 rows x 128 E4M3 codes: one swizzle atom wide
+    // d = 64, 128: two 128-row query tiles per CTA; d = 256: one (the O
+    // accumulator takes 256 TMEM columns)
+    static constexpr int NQ = D <= 128 ? 2 : 1;
+    static constexpr int NSK = D == 256 ? 3 : 6, NSV = D == 256 ? 2 : 4;
+    // rows of E4M3 codes in swizzle atoms of 128 bytes (d = 64: 64 bytes, the
+    // 64-byte swizzle); a 128-row tile is D / kRowBytes atoms kAtom apart
+    static constexpr int kRowBytes = D < 128 ? D : 128;
+    static constexpr int kAtom = 128 * kRowBytes;
+    static constexpr int kTileBytes = 128 * D;
     static constexpr int kOChunk = 128 * 128;           // 64 16-bit columns of a 128-row O tile
     static constexpr int kQOff = 0;
     static constexpr int kKOff = kQOff + NQ * kTileBytes;
@@ -231,32 +240,37 @@ struct Fwd8Cfg {
     static constexpr int kNumBars = kBarMmaDone + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
-    static constexpr int kThreads = 384;
-    static constexpr int kWarpTma = 8, kWarpMma = 9, kWarpTmaV = 10;
-    static constexpr int kRegsSoftmax = 216, kRegsCtl = 72;
-    static constexpr int kOCol = 256;
-    static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= 384 * 168, "register split");
-    static_assert(NQ * 2 * kOChunk <= NSK * kTileBytes, "O staging fits the K ring");
+    static constexpr int kSoftmaxWarps = 4 * NQ;
+    // softmax warpgroups, then one of TMA (K), MMA, TMA (V) and an idle warp
+    static constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
+    static constexpr int kWarpTma = kSoftmaxWarps, kWarpMma = kSoftmaxWarps + 1, kWarpTmaV = kSoftmaxWarps + 2;
+    static constexpr int kRegsSoftmax = 216, kRegsCtl = 72;   // NQ = 2 only (setmaxnreg)
+    static constexpr int kOCol = 128 * NQ;
+    static_assert(NQ == 1 || 2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= 384 * 168, "register split");
+    static_assert(NQ * (D / 64) * kOChunk <= NSK * kTileBytes, "O staging fits the K ring");
+    static_assert(kOCol + NQ * D <= 512, "TMEM columns");
+    static_assert(D == 64 || D == 128 || D == 256, "head dim");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 // Key blocks of a causal or dense square problem seen by query block pair (rb0, rb0 + 1):
 // j < min(nb, rb0 + 2) (causal) or j < nb; flags bit t: block j is seen by tile t.
+template <int NQ>
 __device__ __forceinline__ uint32_t fwd8_flags(const Fwd8Params &p, int rb0, int j) {
     uint32_t f = 0;
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < NQ; ++t)
         if (rb0 + t < p.nb && (!p.causal || j <= rb0 + t)) f |= 1u << t;
     return f;
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(384, 1)
+template <int D, bool BF16>
+__global__ void __launch_bounds__(Fwd8Cfg<D>::kThreads, 1)
     fwd8_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                 const Fwd8Params p) {
-    using C = Fwd8Cfg;
-    constexpr int D = C::D, NQ = C::NQ, NSK = C::NSK, NSV = C::NSV;
+    using C = Fwd8Cfg<D>;
+    constexpr int NQ = C::NQ, NSK = C::NSK, NSV = C::NSV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -308,8 +322,8 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp >= 8) {
-        setmaxnreg_dec<C::kRegsCtl>();
+    if (warp >= C::kSoftmaxWarps) {
+        if constexpr (NQ == 2) setmaxnreg_dec<C::kRegsCtl>();
         if (warp == C::kWarpTma || warp == C::kWarpTmaV) {
             // ------------------------------------------------------------ producers
             const bool do_k = warp == C::kWarpTma;
@@ -319,7 +333,9 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
                 for (int t = 0; t < NQ; ++t)
                     if (rb0 + t < p.nb)
-                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes, &tmq, bar(C::kBarQ), 0, (rb0 + t) * 128, bh);
+                        for (int a = 0; a < D / C::kRowBytes; ++a)
+                            tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + a * C::kAtom, &tmq, bar(C::kBarQ),
+                                        a * C::kRowBytes, (rb0 + t) * 128, bh);
             }
             __syncwarp();
             const int NS = do_k ? NSK : NSV;
@@ -333,7 +349,9 @@ __global__ void __launch_bounds__(384, 1)
                 if (!wait_bar(bar(empty0 + s), ((n / NS) & 1) ^ 1u, abort_flag)) break;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar(full0 + s), C::kTileBytes);
-                    tma_load_3d(sbase + off0 + s * C::kTileBytes, map, bar(full0 + s), 0, j * 128, bh);
+                    for (int a = 0; a < D / C::kRowBytes; ++a)
+                        tma_load_3d(sbase + off0 + s * C::kTileBytes + a * C::kAtom, map, bar(full0 + s),
+                                    a * C::kRowBytes, j * 128, bh);
                 }
                 __syncwarp();
             }
@@ -344,28 +362,37 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t leader = elect_one();
             constexpr uint32_t kIdS = instr_desc_e4m3(128, 128, false, false);
             constexpr uint32_t kIdO = instr_desc_e4m3(128, D, false, true);
-            const SmemDesc dQ = make_desc(sbase + C::kQOff, 16, 1024);
-            const SmemDesc dK = make_desc(sbase + C::kKOff, 16, 1024);
-            const SmemDesc dV = make_desc(sbase + C::kVOff, C::kTileBytes, 1024);
-            auto issue_s = [&](int t, int s) {   // S_t = Q8_t K8_j^T: four K = 32 steps along the 128-byte rows
+            // 8-row groups of the swizzle atoms are 8 rows apart (sbo); V8 is the
+            // MN-major B operand of P V, its atoms along d kAtom apart (lbo)
+            constexpr uint32_t kSbo = 8 * C::kRowBytes;
+            auto desc = [&](uint32_t a, uint32_t lbo) { return D == 64 ? make_desc_sw64(a, lbo, kSbo) : make_desc(a, lbo, kSbo); };
+            const SmemDesc dQ = desc(sbase + C::kQOff, 16);
+            const SmemDesc dK = desc(sbase + C::kKOff, 16);
+            const SmemDesc dV = desc(sbase + C::kVOff, C::kAtom);
+            auto issue_s = [&](int t, int s) {   // S_t = Q8_t K8_j^T: K = 32 steps along the rows of each atom
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    mma8_ss(tmem + 128u * t, dQ.at(t * C::kTileBytes + 32 * k), dK.at(s * C::kTileBytes + 32 * k), kIdS,
+                for (int k = 0; k < D / 32; ++k) {
+                    constexpr int kSteps = C::kRowBytes / 32;   // K steps per atom
+                    const uint32_t o = (k / kSteps) * C::kAtom + 32 * (k % kSteps);
+                    mma8_ss(tmem + 128u * t, dQ.at(t * C::kTileBytes + o), dK.at(s * C::kTileBytes + o), kIdS,
                             k > 0 ? 1u : 0u, leader);
+                }
             };
             auto issue_pv = [&](int t, int s, bool acc) {   // O_t += P8_t V8_j: keys 32k.. in P8 columns 8k..
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma8_ts(tmem + C::kOCol + D * t, tmem + 128u * t + 8u * k, dV.at(s * C::kTileBytes + k * 4096), kIdO,
-                            (acc || k > 0) ? 1u : 0u, leader);
+                    mma8_ts(tmem + C::kOCol + D * t, tmem + 128u * t + 8u * k,
+                            dV.at(s * C::kTileBytes + k * 32 * C::kRowBytes), kIdO, (acc || k > 0) ? 1u : 0u, leader);
             };
-            int cnt[NQ] = {0, 0};
+            int cnt[NQ];
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) cnt[t] = 0;
             bool ok = true;
             if (nkb > 0) {
                 ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag);
                 if (ok) {
                     tc_fence_after();
-                    const uint32_t f = fwd8_flags(p, rb0, 0);
+                    const uint32_t f = fwd8_flags<NQ>(p, rb0, 0);
                     for (int t = 0; t < NQ; ++t)
                         if ((f >> t) & 1u) {
                             issue_s(t, 0);
@@ -378,8 +405,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int u = 0; ok && u < nkb; ++u) {
                 const int s = u % NSV;
                 const bool have_n = u + 1 < nkb;
-                const uint32_t f = fwd8_flags(p, rb0, u);
-                const uint32_t fn = have_n ? fwd8_flags(p, rb0, u + 1) : 0u;
+                const uint32_t f = fwd8_flags<NQ>(p, rb0, u);
+                const uint32_t fn = have_n ? fwd8_flags<NQ>(p, rb0, u + 1) : 0u;
                 const int sn = (u + 1) % NSK;
                 ok = wait_bar(bar(C::kBarVFull + s), (u / NSV) & 1, abort_flag);
                 if (!ok) break;
@@ -417,7 +444,7 @@ __global__ void __launch_bounds__(384, 1)
             drain_bar(bar(C::kBarMmaDone), 0);
         }
     } else {
-        setmaxnreg_inc<C::kRegsSoftmax>();
+        if constexpr (NQ == 2) setmaxnreg_inc<C::kRegsSoftmax>();
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int wq = warp & 3;
@@ -432,7 +459,7 @@ __global__ void __launch_bounds__(384, 1)
         int cnt = 0;
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            if (!((fwd8_flags(p, rb0, j) >> t) & 1u)) continue;
+            if (!((fwd8_flags<NQ>(p, rb0, j) >> t) & 1u)) continue;
             const float c = cq * p.sk[static_cast<size_t>(bh) * p.nb + j];   // score -> base-2 logit of this tile pair
             ok = wait_bar(bar(C::kBarSFull + t), cnt & 1, abort_flag);
             if (!ok) break;
@@ -514,7 +541,7 @@ __global__ void __launch_bounds__(384, 1)
         // O_t (16-bit) staged in the finished K ring as 128-byte-swizzled
         // 64-column chunks, then written by TMA stores (rows >= N clipped)
         const bool epi = rb < p.nb && ok;
-        uint8_t *stage = smem + C::kKOff + t * 2 * C::kOChunk;
+        uint8_t *stage = smem + C::kKOff + t * (D / 64) * C::kOChunk;
         if (epi) {
             const float sv_h = p.sv[static_cast<size_t>(bh) * p.nb];
             const float inv_l = (cnt > 0 && l_r > 0.f) ? sv_h / l_r : 0.0f;

@@ -238,11 +238,11 @@ FA_API int fa_bwd_noalloc(const void *q, const void *k, const void *v, const voi
  * Three launches on `stream`.  Pointers: the tensors 16-byte aligned, the
  * scales and signs 4-byte aligned.
  *
- * fa_fwd_fp8: the forward on those codes (d = 128 only, N = Nq = Nk, causal or
- * dense, no mask): S = scale * sq * sk * q8 . k8 with fp32 accumulation, the
- * online softmax in fp32, P rounded to E4M3 for the P V product,
+ * fa_fwd_fp8: the forward on those codes (d = 64, 128 or 256, N = Nq = Nk, causal
+ * or dense, no mask): S = scale * sq * sk * q8 . k8 with fp32 accumulation,
+ * the online softmax in fp32, P rounded to E4M3 for the P V product,
  * O = sv * sum P8 v8 / sum P8 written as out_dtype (FA_F16/FA_BF16) [B][H][N][d],
- * lse [B][H][N] fp32 as fa_fwd.  Returns FA_ERR_UNSUPPORTED for d != 128.
+ * lse [B][H][N] fp32 as fa_fwd.  Returns FA_ERR_UNSUPPORTED for other d.
  */
 FA_API int fa_fp8_quantize_qkv(const void *q, const void *k, const void *v,
                                uint8_t *q8, uint8_t *k8, uint8_t *v8,

@@ -105,8 +105,9 @@ def _o_bar(codes, bh, rows, causal, scale, o_ref):
 @pytest.mark.parametrize("N", [1, 129, 300, 1000])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_fp8_forward_parity(N, causal, dtype):
-    B, H, d = 1, 2, 128
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_fp8_forward_parity(N, causal, dtype, d):
+    B, H = 1, 2
     q, k, v, _ = inputs.make_qkv(B, H, N, d, dtype, seed=7 + N, with_dout=False)
     signs = inputs.hadamard_signs(d, seed=2)
     codes, o, lse = _fp8_run(q, k, v, causal, signs)
@@ -122,8 +123,9 @@ def test_fp8_forward_parity(N, causal, dtype):
         assert np.all(err <= bar), (bh, float(err.max()), float((err / bar).max()))
 
 
-def test_fp8_identical_v_rows_exact():
-    B, H, N, d = 1, 2, 700, 128
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_fp8_identical_v_rows_exact(d):
+    B, H, N = 1, 2, 700
     q, k, v, _ = inputs.make_qkv(B, H, N, d, "bf16", seed=3, with_dout=False)
     v = v[:, :, :1].expand(B, H, N, d).contiguous()
     codes, o, _ = _fp8_run(q, k, v, True)
@@ -135,9 +137,10 @@ def test_fp8_identical_v_rows_exact():
     assert np.abs(got - want16[:, :, None, :]).max() <= 1e-2 * np.abs(want).max()
 
 
-def test_fp8_dsweep_shape_sampled():
-    # B=4 H=16 N=4096 d=128 causal: sampled rows per head against the oracle on the GPU's codes
-    B, H, N, d = 4, 16, 4096, 128
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_fp8_dsweep_shape_sampled(d):
+    # B=4 H=16 N=4096 causal: sampled rows per head against the oracle on the GPU's codes
+    B, H, N = 4, 16, 4096
     q, k, v, _ = inputs.make_qkv(B, H, N, d, "bf16", seed=0, with_dout=False)
     codes, o, lse = _fp8_run(q, k, v, True, inputs.hadamard_signs(d, seed=0))
     o = o.reshape(B * H, N, d)
