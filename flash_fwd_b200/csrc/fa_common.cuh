@@ -546,12 +546,12 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
     return r;
 }
 
-// max(a, b, c) in one instruction
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
+// max(a, b, c) as two two-input maxima.  (The three-input max.f32 written as
+// inline PTX gave wrong row maxima in the softmax of one build: on rows whose
+// 128 scores were all -inf, two of its four chains returned +0.0 and a value
+// of the order of 2^-125, while a two-input fmaxf chain over the same
+// registers returned -inf.)
+__device__ __forceinline__ float fmax3(float a, float b, float c) { return fmaxf(a, fmaxf(b, c)); }
 
 // 2^x for a pair, on the FMA pipe: x = j + f with j = round(x) (by adding
 // 1.5 * 2^23, whose fp32 ulp is 1) and f in [-1/2, 1/2]; 2^f from the
