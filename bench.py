@@ -64,11 +64,22 @@ WORKLOADS = {
     "fp8_128": dict(B=4, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
     "fp8_64": dict(B=4, H=16, N=4096, d=64, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
     "fp8_256": dict(B=4, H=16, N=4096, d=256, dtype="bf16", causal=True, sparse=False, bwd=False, fp8=True),
+    # a packed variable-length batch (fa_fwd_varlen / fa_bwd_varlen): 16
+    # sequences with lengths drawn uniformly from [512, 4096] (seeded), N = the
+    # bound of the lengths (max_seqlen)
+    "varlen128": dict(B=16, H=16, N=4096, d=128, dtype="bf16", causal=True, sparse=False, bwd=True,
+                      varlen=(512, 4096)),
 }
 
 
 def general(w):
     return "Nk" in w or "window" in w or w.get("alibi", False)
+
+
+def varlen_lengths(w):
+    """The sequence lengths of a packed workload (seed 0: every rank the same mix)."""
+    from flash_fwd_b200 import inputs
+    return inputs.varlen_lengths(w["B"], w["varlen"][0], w["varlen"][1], seed=0)
 
 
 L2_BYTES = 126 * 1024 * 1024
@@ -99,7 +110,9 @@ def peaks():
 
 def workload_flops(w, kept_blocks=None):
     from flash_fwd_b200 import accounting as acc
-    if w["sparse"]:
+    if w.get("varlen"):
+        f = sum(acc.fwd_flops(1, w["H"], n, w["d"], w["causal"]) for n in varlen_lengths(w))
+    elif w["sparse"]:
         f = acc.sparse_fwd_flops(w["B"], w["H"], w["d"], kept_blocks)
     elif "Nk" in w or "window" in w:
         f = acc.general_fwd_flops(w["B"], w["H"], w["N"], w.get("Nk", w["N"]), w["d"], w["causal"], w.get("window"))
@@ -119,6 +132,10 @@ def describe(name, w):
     s += " fwd+bwd" if w["bwd"] else " fwd"
     s += " (deterministic backward)" if w.get("deterministic") else ""
     s += " (FP8 E4M3 with Hadamard rotation; step = quantise + forward)" if w.get("fp8") else ""
+    if w.get("varlen"):
+        n = varlen_lengths(w)
+        s += (f" (packed variable-length batch: {len(n)} sequences, lengths uniform in "
+              f"[{w['varlen'][0]}, {w['varlen'][1]}], {sum(n)} tokens, max_seqlen {max(n)})")
     return s
 
 
@@ -231,6 +248,20 @@ def make_inputs(w, seed, device):
     import torch
 
     from flash_fwd_b200 import inputs
+    if w.get("varlen"):
+        import flash_fwd_b200 as fa
+        n = varlen_lengths(w)
+        cu_q, cu_k, q, k, v, do = inputs.make_varlen(n, n, w["H"], w["d"], w["dtype"], seed=seed)
+        host = dict(q=q, k=k, v=v, do=do, cu_q=cu_q, cu_k=cu_k, mask=None, slopes=None)
+        dev = {x: (y.to(device) if y is not None else None) for x, y in host.items()}
+        dev["o"] = torch.empty_like(dev["q"])
+        dev["lse"] = torch.empty((w["H"], q.shape[0]), dtype=torch.float32, device=device)
+        dev["dq"] = torch.empty_like(dev["q"])
+        dev["dk"], dev["dv"] = torch.empty_like(dev["k"]), torch.empty_like(dev["v"])
+        dev["ws"] = torch.empty(fa.fa_bwd_varlen_workspace_bytes(w["B"], w["H"], q.shape[0], max(n), w["d"]),
+                                dtype=torch.uint8, device=device)
+        dev["max_n"] = max(n)
+        return host, dev
     if "Nk" in w:
         q, k, v, do = inputs.make_qkv_cross(w["B"], w["H"], w["N"], w["Nk"], w["d"], w["dtype"], seed=seed)
     else:
@@ -256,7 +287,12 @@ def make_inputs(w, seed, device):
 def step(w, t, stream):
     import flash_fwd_b200 as fa
     scale = 1.0 / w["d"] ** 0.5
-    if w.get("fp8"):
+    if w.get("varlen"):
+        fa.fa_fwd_varlen(t["q"], t["k"], t["v"], t["o"], t["lse"], t["cu_q"], t["cu_k"], t["max_n"], t["max_n"],
+                         w["causal"], scale, stream=stream)
+        fa.fa_bwd_varlen(t["q"], t["k"], t["v"], t["o"], t["do"], t["lse"], t["dq"], t["dk"], t["dv"], t["ws"],
+                         t["cu_q"], t["cu_k"], t["max_n"], t["max_n"], w["causal"], scale, stream=stream)
+    elif w.get("fp8"):
         q8, k8, v8, sq, sk, sv = fa.fa_fp8_quantize_qkv(t["q"], t["k"], t["v"], t["signs"], stream)
         fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, t["o"], t["lse"], w["causal"], scale, stream)
     elif w.get("deterministic"):
@@ -295,6 +331,11 @@ def oracle_head_pass(host, w, head):
     N, Nk, d = w["N"], w.get("Nk", w["N"]), w["d"]
     b, h = divmod(head, w["H"])
     sl = lambda t, n: t[b, h].reshape(1, n, d).double().numpy()  # noqa: E731
+    if w.get("varlen"):
+        # sequence b, head h of the packed batch: its own square problem
+        c0, c1 = int(host["cu_q"][b]), int(host["cu_q"][b + 1])
+        N = Nk = c1 - c0
+        sl = lambda t, n: t[c0:c1, h].reshape(1, n, d).double().numpy()  # noqa: E731
     Q, K, V = sl(host["q"], N), sl(host["k"], Nk), sl(host["v"], Nk)
     flags = (oracle.CAUSAL if w["causal"] else 0) | (oracle.SPARSE if w["sparse"] else 0)
     mask = host["mask"].numpy() if w["sparse"] else None
@@ -326,17 +367,27 @@ def per_head_flops(w, kept_blocks):
     return (f + b) / (w["B"] * w["H"])
 
 
+def head_flops(w, kept_blocks, head):
+    """FLOPs of (batch, head) pair number `head` (a packed batch's sequences differ)."""
+    if not w.get("varlen"):
+        return per_head_flops(w, kept_blocks)
+    from flash_fwd_b200 import accounting as acc
+    n = varlen_lengths(w)[head // w["H"]]
+    return (3.5 if w["bwd"] else 1.0) * acc.fwd_flops(1, 1, n, w["d"], w["causal"])
+
+
 def cpu_sample(host, w, kept_blocks, budget_s, max_heads=None):
     """Whole (batch, head) passes of the oracle until the budget is spent (at
     least one).  Returns (heads, seconds, TFLOP/s, forward s, backward s)."""
     heads = w["B"] * w["H"] if max_heads is None else min(max_heads, w["B"] * w["H"])
-    done, tf, tb = 0, 0.0, 0.0
+    done, tf, tb, fl = 0, 0.0, 0.0, 0.0
     while done < heads and (tf + tb < budget_s or done == 0):
         f, b = oracle_head_pass(host, w, done)
         tf, tb = tf + f, tb + b
+        fl += head_flops(w, kept_blocks, done)
         done += 1
     secs = tf + tb
-    return done, secs, done * per_head_flops(w, kept_blocks) / secs / 1e12, tf, tb
+    return done, secs, fl / secs / 1e12, tf, tb
 
 
 def oracle_seconds(w, heads, tf, tb):
@@ -356,12 +407,14 @@ def run_reference(args, w, name):
     kept = int(host["mask"].sum()) if w["sparse"] else None
     for i in range(args.warmup):
         oracle_head_pass(host, w, i % (w["B"] * w["H"]))
-    tf = tb = 0.0
+    tf = tb = fl = 0.0
     for i in range(args.steps):
-        f, b = oracle_head_pass(host, w, (args.warmup + i) % (w["B"] * w["H"]))
+        head = (args.warmup + i) % (w["B"] * w["H"])
+        f, b = oracle_head_pass(host, w, head)
         tf, tb = tf + f, tb + b
+        fl += head_flops(w, kept, head)
     secs = tf + tb
-    val = args.steps * per_head_flops(w, kept) / secs / 1e12
+    val = fl / secs / 1e12
     cores = os.cpu_count()
     what = ("E4M3 quantisation and the FP8 forward on all rows" if w.get("fp8") else
             "forward on all rows, dQ on all rows, dK/dV on all keys" if w["bwd"] else "forward on all rows")
@@ -380,6 +433,10 @@ def run_reference(args, w, name):
 
 def make_inputs_cpu(w):
     from flash_fwd_b200 import inputs
+    if w.get("varlen"):
+        n = varlen_lengths(w)
+        cu_q, cu_k, q, k, v, do = inputs.make_varlen(n, n, w["H"], w["d"], w["dtype"], seed=0)
+        return dict(q=q, k=k, v=v, do=do, cu_q=cu_q, cu_k=cu_k, mask=None, slopes=None), None
     if "Nk" in w:
         q, k, v, do = inputs.make_qkv_cross(w["B"], w["H"], w["N"], w["Nk"], w["d"], w["dtype"], seed=0)
     else:
@@ -581,7 +638,7 @@ def run_ours(args, w, name):
     # ---------------- end to end through host buffers
     e2e = None
     if args.e2e_steps > 0:
-        pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "do") if host[n] is not None}
+        pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "do", "cu_q", "cu_k") if host.get(n) is not None}
         outs = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True)
                 for n in (["o", "lse", "dq", "dk", "dv"] if w["bwd"] else ["o", "lse"])}
         h2d = sum(x.numel() * x.element_size() for x in pin.values())

@@ -17,7 +17,8 @@ __all__ = [
     "fa_version", "attention_fwd", "attention_bwd", "FA_BLOCK", "fa_profile_enable", "fa_profile_read",
     "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes", "fa_bwd_deterministic",
     "fa_bwd_deterministic_workspace_bytes", "fa_fp8_quantize_qkv", "fa_fwd_fp8", "attention_fwd_fp8",
-    "fa_bwd_noalloc",
+    "fa_bwd_noalloc", "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_bytes", "attention_fwd_varlen",
+    "attention_bwd_varlen",
 ]
 
 FA_BLOCK = 128
@@ -64,6 +65,10 @@ def load_library():
     lib.fa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, vp, i, vp]
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [i, i, i, i, f, i, i, vp]
+    lib.fa_fwd_varlen.argtypes = [vp] * 7 + [i] * 7 + [f, i, i, i, vp, i, vp]
+    lib.fa_bwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_varlen_workspace_bytes.restype = sz
+    lib.fa_bwd_varlen.argtypes = [vp] * 10 + [sz, vp, vp] + [i] * 7 + [f, i, i, i, vp, i, vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -73,6 +78,7 @@ def load_library():
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
                lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8, lib.fa_bwd_noalloc,
+               lib.fa_fwd_varlen, lib.fa_bwd_varlen,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -392,3 +398,91 @@ def attention_fwd_fp8(q, k, v, causal=False, scale=None, signs=None, stream=None
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     fa_fwd_fp8(q8, k8, v8, sq, sk, sv, o, lse, causal, scale, stream)
     return o, lse
+
+
+# ---------------------------------------------------------------- packed variable-length batches
+_I32 = (torch.int32,)
+
+
+def _need_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dout=None, dq=None,
+                 dk=None, dv=None, workspace=None, alibi_slopes=None):
+    """Checks the tensors of one packed call; returns (B, H, total_q, total_k, d)."""
+    dev = _current_device() if isinstance(q, torch.Tensor) and q.is_cuda else -1
+    _need("q", q, dev, _HALF)
+    if q.dim() != 3:
+        raise ValueError("packed q, k, v: expected [total, H, d] tensors")
+    total_q, H, d = (int(x) for x in q.shape)
+    _need("k", k, dev, (q.dtype,))
+    if k.dim() != 3 or int(k.shape[1]) != H or int(k.shape[2]) != d:
+        raise ValueError(f"k: shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    total_k = int(k.shape[0])
+    _need("v", v, dev, (q.dtype,), shape=k.shape)
+    _need("o", o, dev, (q.dtype,), shape=q.shape)
+    _need("lse", lse, dev, _F32, shape=(H, total_q))
+    _need("cu_seqlens_q", cu_seqlens_q, dev, _I32)
+    _need("cu_seqlens_k", cu_seqlens_k, dev, _I32, shape=cu_seqlens_q.shape)
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens: expected [B + 1] int32 tensors")
+    B = cu_seqlens_q.numel() - 1
+    for name, t, like in (("dout", dout, q), ("dq", dq, q), ("dk", dk, k), ("dv", dv, k)):
+        if t is not None:
+            _need(name, t, dev, (q.dtype,), shape=like.shape)
+    if workspace is not None:
+        _need("workspace", workspace, dev)
+    if alibi_slopes is not None:
+        _need("alibi_slopes", alibi_slopes, dev, _F32, numel=H)
+    return B, H, total_q, total_k, d
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                  scale=None, window=None, alibi_slopes=None, stream=None):
+    """Forward of a packed batch: q, o [total_q, H, d]; k, v [total_k, H, d]; lse [H, total_q] fp32;
+    cu_seqlens_q / _k int32 [B + 1] on the device; max_seqlen_* host ints bounding the lengths."""
+    B, H, tq, tk, d = _need_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                                   alibi_slopes=alibi_slopes)
+    wl, wr = _window(window)
+    rc = load_library().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                                      _ptr(cu_seqlens_k), B, H, tq, tk, int(max_seqlen_q), int(max_seqlen_k), d,
+                                      _scale(scale, d), int(bool(causal)), wl, wr, _ptr(alibi_slopes), _dtype(q),
+                                      _stream(stream))
+    _check(rc, "fa_fwd_varlen")
+
+
+def fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_q, d):
+    return load_library().fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_q, d)
+
+
+def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                  max_seqlen_k, causal=False, scale=None, window=None, alibi_slopes=None, stream=None):
+    B, H, tq, tk, d = _need_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dout,
+                                   dq, dk, dv, workspace, alibi_slopes)
+    wl, wr = _window(window)
+    rc = load_library().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, tq, tk, int(max_seqlen_q),
+                                      int(max_seqlen_k), d, _scale(scale, d), int(bool(causal)), wl, wr,
+                                      _ptr(alibi_slopes), _dtype(q), _stream(stream))
+    _check(rc, "fa_bwd_varlen")
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False, scale=None,
+                         window=None, alibi_slopes=None, stream=None):
+    """Allocates O [total_q, H, d] and LSE [H, total_q] and runs the packed forward; returns (o, lse)."""
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, scale, window,
+                  alibi_slopes, stream)
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                         causal=False, scale=None, window=None, alibi_slopes=None, workspace=None, stream=None):
+    """Allocates dQ, dK, dV (and the workspace unless given) and runs the packed backward."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        nbytes = fa_bwd_varlen_workspace_bytes(cu_seqlens_q.numel() - 1, int(q.shape[1]), int(q.shape[0]),
+                                               int(max_seqlen_q), int(q.shape[2]))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                  max_seqlen_k, causal, scale, window, alibi_slopes, stream)
+    return dq, dk, dv

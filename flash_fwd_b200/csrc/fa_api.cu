@@ -87,6 +87,25 @@ int make_map(CUtensorMap *map, const void *base, int d, int N, long long BH, int
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// Packed [total][H][d] 16-bit tensor (variable-length batches) seen as a 3-D
+// TMA map {d, total, H}: the same 64 x rows x 1 boxes as make_map, with the
+// row coordinate running over the packed rows of one head (stride H * d
+// elements) and the plane over heads (stride d).
+int make_map_packed(CUtensorMap *map, const void *base, int d, int total, int H, int dtype, int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return FA_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(total), static_cast<cuuint64_t>(H)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // [BH][N][d] E4M3 codes as a 3-D TMA map {d, N, BH} with d x 128 x 1 boxes
 // (d = 128: one 128-byte swizzle atom per row); rows past N read as zeros.
 int make_map8(CUtensorMap *map, const void *base, int d, int N, long long BH) {
@@ -142,11 +161,11 @@ int check_problem(const Problem &pr) {
     return FA_OK;
 }
 
-template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL, bool VARLEN = false>
 int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mo,
                const fa::FwdParams &p, int BH, cudaStream_t stream) {
     using C = fa::FwdCfg<D, NQ, NSK, NSV>;
-    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, GENERAL>;
+    auto kern = fa::fwd_kernel<D, NQ, NSK, NSV, BF16, GENERAL, VARLEN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     const long long items = static_cast<long long>(BH) * ((p.nqb + NQ - 1) / NQ);
@@ -169,13 +188,13 @@ int launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <bool BF16, bool GENERAL>
+template <bool BF16, bool GENERAL, bool VARLEN = false>
 int dispatch_fwd(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mo,
                  const fa::FwdParams &p, int BH, cudaStream_t s) {
     switch (d) {
-        case 64: return launch_fwd<64, 2, 6, 4, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
-        case 128: return launch_fwd<128, 2, 3, 2, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
-        case 256: return launch_fwd<256, 1, 1, 1, BF16, GENERAL>(mq, mk, mv, mo, p, BH, s);
+        case 64: return launch_fwd<64, 2, 6, 4, BF16, GENERAL, VARLEN>(mq, mk, mv, mo, p, BH, s);
+        case 128: return launch_fwd<128, 2, 3, 2, BF16, GENERAL, VARLEN>(mq, mk, mv, mo, p, BH, s);
+        case 256: return launch_fwd<256, 1, 1, 1, BF16, GENERAL, VARLEN>(mq, mk, mv, mo, p, BH, s);
         default: return FA_ERR_UNSUPPORTED;
     }
 }
@@ -193,7 +212,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     if ((rc = make_map(&mo, o, pr.d, pr.Nq, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mk, k, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
     if ((rc = make_map(&mv, v, pr.d, pr.Nk, BH, pr.dtype, 128)) != FA_OK) return rc;
-    fa::FwdParams p;
+    fa::FwdParams p{};
     p.lse = lse;
     p.mask = pr.mask;
     p.alibi = pr.alibi;
@@ -216,6 +235,66 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
                        : dispatch_fwd<true, false>(pr.d, mq, mk, mv, mo, p, BH, s);
     return general ? dispatch_fwd<false, true>(pr.d, mq, mk, mv, mo, p, BH, s)
                    : dispatch_fwd<false, false>(pr.d, mq, mk, mv, mo, p, BH, s);
+}
+
+// A packed variable-length batch: B sequences of at most Nq (Nk) query (key)
+// rows, total_q (total_k) packed rows in all, lengths in cu_q / cu_k.
+struct Packed {
+    const int *cu_q, *cu_k;
+    int total_q, total_k;
+};
+
+int check_packed(const Packed &pk, const Problem &pr) {
+    if (!pk.cu_q || !pk.cu_k) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(pk.cu_q) & 3u) || (reinterpret_cast<uintptr_t>(pk.cu_k) & 3u))
+        return FA_ERR_MISALIGNED;
+    if (pk.total_q < 1 || pk.total_k < 1 || pr.Nq > pk.total_q || pr.Nk > pk.total_k) return FA_ERR_INVALID_ARG;
+    if (pr.mask) return FA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(pk.total_q) * pr.H > 0x7fffffffLL ||
+        static_cast<long long>(pk.total_k) * pr.H > 0x7fffffffLL)
+        return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+int fwd_varlen_impl(const void *q, const void *k, const void *v, void *o, float *lse, const Problem &pr,
+                    const Packed &pk, void *stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int rc = check_problem(pr);
+    if (rc != FA_OK) return rc;
+    if ((rc = check_packed(pk, pr)) != FA_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    const int BH = static_cast<int>(pr.BH());
+    if (static_cast<long long>(BH) * ((pr.Nq + 127) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv, mo;
+    if ((rc = make_map_packed(&mq, q, pr.d, pk.total_q, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mo, o, pr.d, pk.total_q, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mk, k, pr.d, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mv, v, pr.d, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    fa::FwdParams p{};
+    p.lse = lse;
+    p.mask = nullptr;
+    p.alibi = pr.alibi;
+    p.Nq = pr.Nq;   // the longest sequences: they size the item grid
+    p.Nk = pr.Nk;
+    p.off = pr.off();
+    p.wl = pr.wl();
+    p.wr = pr.wr();
+    p.nqb = (pr.Nq + 127) / 128;
+    p.nkb = (pr.Nk + 127) / 128;
+    p.nbh = BH;
+    p.H = pr.H;
+    p.mode = pr.mode();
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * kLog2e;
+    p.cu_q = pk.cu_q;
+    p.cu_k = pk.cu_k;
+    p.o = o;
+    p.total_q = pk.total_q;
+    p.total_k = pk.total_k;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pr.dtype == FA_BF16) return dispatch_fwd<true, true, true>(pr.d, mq, mk, mv, mo, p, BH, s);
+    return dispatch_fwd<false, true, true>(pr.d, mq, mk, mv, mo, p, BH, s);
 }
 
 
@@ -377,6 +456,112 @@ int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, vo
     return general ? dispatch_bwd<false, true>(bb, pr, det, s) : dispatch_bwd<false, false>(bb, pr, det, s);
 }
 
+// ---------------------------------------------------------------- packed batches
+// Workspace of the packed backward: lse2 and D [BH][Npad] (Npad = the longest
+// query sequence rounded up to 128), then the fp32 dQ accumulator
+// [H][total_q][d].
+size_t bwd_varlen_workspace_bytes(long long BH, int H, int total_q, int max_nq, int d) {
+    return 2 * static_cast<size_t>(BH) * fa::bwd_npad(max_nq) * 4 +
+           static_cast<size_t>(H) * static_cast<size_t>(total_q) * d * 4;
+}
+
+template <int D, bool BF16>
+int launch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk, cudaStream_t stream) {
+    using C = fa::BwdCfg<D, D == 64 ? 3 : 2>;
+    constexpr int BM = C::BM;
+    const int BH = static_cast<int>(pr.BH());
+    const int Npad = fa::bwd_npad(pr.Nq);
+    float *lse2 = static_cast<float *>(bb.workspace);
+    float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
+    float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
+    {
+        constexpr int TPR = D / 8;
+        const long long threads = static_cast<long long>(BH) * Npad * TPR;
+        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        ProfScope prof(1, stream);
+        fa::bwd_pre_varlen_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint4 *>(bb.o), static_cast<const uint4 *>(bb.dout), bb.lse, lse2, dvec,
+            reinterpret_cast<float4 *>(dqacc), pk.cu_q, pr.H, pk.total_q, pr.Nq, Npad, BH);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    CUtensorMap mk, mv, mq, mdo, mdk, mdv;
+    int rc;
+    if ((rc = make_map_packed(&mk, bb.k, D, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mdk, bb.dk, D, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mdv, bb.dv, D, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mv, bb.v, D, pk.total_k, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mq, bb.q, D, pk.total_q, pr.H, pr.dtype, BM)) != FA_OK) return rc;
+    if ((rc = make_map_packed(&mdo, bb.dout, D, pk.total_q, pr.H, pr.dtype, BM)) != FA_OK) return rc;
+    fa::BwdParams p{};
+    p.lse2 = lse2;
+    p.dvec = dvec;
+    p.dqacc = dqacc;
+    p.dq = nullptr;
+    p.dk = bb.dk;
+    p.dv = bb.dv;
+    p.mask = nullptr;
+    p.alibi = pr.alibi;
+    p.Nq = pr.Nq;   // the longest sequences
+    p.Nk = pr.Nk;
+    p.off = pr.off();
+    p.wl = pr.wl();
+    p.wr = pr.wr();
+    p.H = pr.H;
+    p.Npad = Npad;
+    p.nkb = (pr.Nk + 127) / 128;
+    p.nqt = (pr.Nq + BM - 1) / BM;
+    p.nbh = BH;
+    p.mode = pr.mode();
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * kLog2e;
+    p.cu_q = pk.cu_q;
+    p.cu_k = pk.cu_k;
+    p.total_q = pk.total_q;
+    p.total_k = pk.total_k;
+    auto kern = fa::bwd_kernel<D, D == 64 ? 3 : 2, BF16, true, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    {
+        // B x H x (key blocks of the longest sequence); CTAs past their own
+        // sequence's keys return at once
+        const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb));
+        ProfScope prof(2, stream);
+        kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, mdk, mdv, p);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    {
+        const long long n8 = static_cast<long long>(pr.H) * pk.total_q * (D / 8);
+        const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+        ProfScope prof(3, stream);
+        fa::bwd_post_varlen_kernel<D, BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(dqacc),
+                                                                         static_cast<uint4 *>(bb.dq), pr.scale,
+                                                                         pr.H, pk.total_q);
+    }
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int bwd_varlen_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, const Packed &pk,
+                    void *stream) {
+    if (!bb.q || !bb.k || !bb.v || !bb.o || !bb.dout || !bb.lse || !bb.dq || !bb.dk || !bb.dv)
+        return FA_ERR_INVALID_ARG;
+    int rc = check_problem(pr);
+    if (rc != FA_OK) return rc;
+    if ((rc = check_packed(pk, pr)) != FA_OK) return rc;
+    if (pr.d == 256) return FA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {bb.q, bb.k, bb.v, bb.o, bb.dout, bb.lse, bb.dq, bb.dk, bb.dv};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+    if (pr.BH() * ((pr.Nk + 127LL) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
+    if (pr.BH() * fa::bwd_npad(pr.Nq) * (pr.d / 8) > 0x7fffffffLL * 256LL) return FA_ERR_UNSUPPORTED;
+    const size_t need = bwd_varlen_workspace_bytes(pr.BH(), pr.H, pk.total_q, pr.Nq, pr.d);
+    if (!bb.workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (!aligned16(bb.workspace)) return FA_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pr.dtype == FA_BF16)
+        return pr.d == 64 ? launch_bwd_varlen<64, true>(bb, pr, pk, s) : launch_bwd_varlen<128, true>(bb, pr, pk, s);
+    return pr.d == 64 ? launch_bwd_varlen<64, false>(bb, pr, pk, s) : launch_bwd_varlen<128, false>(bb, pr, pk, s);
+}
+
 // ---------------------------------------------------------------- fa_bwd_noalloc
 // Scratch for fa_bwd_noalloc, resident on every device that loads the library.
 // Host code must not use this name as a pointer: on the host it is only a
@@ -534,6 +719,34 @@ FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float
                      const float *alibi_slopes, const uint8_t *block_mask, int dtype, void *stream) {
     const Problem pr{B, H, Nq, Nk, d, scale, causal, window_left, window_right, alibi_slopes, block_mask, dtype};
     return fwd_impl(q, k, v, o, lse, pr, stream);
+}
+
+FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                         const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                         int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal, int window_left,
+                         int window_right, const float *alibi_slopes, int dtype, void *stream) {
+    const Problem pr{B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, window_left, window_right, alibi_slopes,
+                     nullptr, dtype};
+    const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+    return fwd_varlen_impl(q, k, v, o, lse, pr, pk, stream);
+}
+
+FA_API size_t fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d) {
+    if (B < 1 || H < 1 || total_q < 1 || max_seqlen_q < 1 || max_seqlen_q > total_q || (d != 64 && d != 128))
+        return 0;
+    return bwd_varlen_workspace_bytes(static_cast<long long>(B) * H, H, total_q, max_seqlen_q, d);
+}
+
+FA_API int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                         const float *lse, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                         const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                         int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal, int window_left,
+                         int window_right, const float *alibi_slopes, int dtype, void *stream) {
+    const Problem pr{B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, window_left, window_right, alibi_slopes,
+                     nullptr, dtype};
+    const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    return bwd_varlen_impl(bb, workspace_bytes, pr, pk, stream);
 }
 
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -61,6 +61,14 @@ struct BwdParams {
     int mode;
     float scale;
     float scale_log2;
+    // packed variable-length batches (VARLEN kernels): sequence b owns packed
+    // rows cu_q[b] .. cu_q[b+1]-1 of q, o, dout, dq and cu_k[b] .. cu_k[b+1]-1
+    // of k, v, dk, dv ([rows][H][D]); lse is [H][total_q], lse2 and dvec are
+    // [BH][Npad] per (sequence, head) and dqacc is [H][total_q][D].  Nq and
+    // Nk above then bound the sequence lengths.
+    const int *cu_q;
+    const int *cu_k;
+    int total_q, total_k;
 };
 
 // ---------------------------------------------------------------------------
@@ -120,6 +128,80 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4 *__restrict_
     const float4 a = acc[2 * i], b = acc[2 * i + 1];
     dq[i] = make_uint4(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale),
                        pack2<BF16>(b.x * scale, b.y * scale), pack2<BF16>(b.z * scale, b.w * scale));
+}
+
+// ---------------------------------------------------------------------------
+// bwd_pre / bwd_post of packed variable-length batches: O, dO, dQ are packed
+// [total_q][H][D], lse [H][total_q]; the statistics go to the padded
+// [BH][Npad] layout of the key-block kernel (rows past a sequence's end:
+// LSE * log2 e = +inf, D = 0, so that they add nothing), the accumulator is
+// [H][total_q][D].
+// ---------------------------------------------------------------------------
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+    bwd_pre_varlen_kernel(const uint4 *__restrict__ o, const uint4 *__restrict__ dout, const float *__restrict__ lse,
+                          float *__restrict__ lse2, float *__restrict__ dvec, float4 *__restrict__ dqacc,
+                          const int *__restrict__ cu_q, int H, int total_q, int max_nq, int Npad, long long BH) {
+    constexpr int TPR = D / 8;   // threads per row, 8 elements (16 bytes) each
+    const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long prow = tid / TPR;                 // padded row index bh * Npad + n
+    const int part = static_cast<int>(tid % TPR);
+    const long long bh = prow / Npad;
+    const int n = static_cast<int>(prow % Npad);
+    SeqSpan sq{0, 0};
+    int h = 0;
+    if (bh < BH) {
+        const int b = static_cast<int>(bh / H);
+        h = static_cast<int>(bh - static_cast<long long>(b) * H);
+        sq = seq_span(cu_q, b, total_q, max_nq);
+    }
+    const bool valid = bh < BH && n < sq.len;
+    const long long t = sq.start + n;                // packed row
+    float acc = 0.f;
+    if (valid) {
+        const long long row = t * H + h;
+        const uint4 a = o[row * TPR + part];
+        const uint4 b = dout[row * TPR + part];
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 x = unpack2<BF16>(av[k]), y = unpack2<BF16>(bv[k]);
+            acc = fmaf(x.x, y.x, acc);
+            acc = fmaf(x.y, y.y, acc);
+        }
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        const long long arow = static_cast<long long>(h) * total_q + t;
+        dqacc[(arow * D + part * 8) / 4] = z;
+        dqacc[(arow * D + part * 8) / 4 + 1] = z;
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (bh < BH && part == 0) {
+        float l2 = INFINITY;      // P = 2^(s - inf) = 0 for rows past the sequence or with no visible key
+        if (valid) {
+            const float L = lse[static_cast<long long>(h) * total_q + t];
+            if (L != -INFINITY) l2 = L * 1.4426950408889634f;
+        }
+        lse2[prow] = l2;
+        dvec[prow] = valid ? acc : 0.f;
+    }
+}
+
+// dq [total_q][H][D] = scale * dqacc [H][total_q][D], 8 elements per thread
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_post_varlen_kernel(const float4 *__restrict__ acc, uint4 *__restrict__ dq,
+                                                              float scale, int H, int total_q) {
+    constexpr int TPR = D / 8;
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;   // over [H][total_q][TPR]
+    if (i >= static_cast<long long>(H) * total_q * TPR) return;
+    const int part = static_cast<int>(i % TPR);
+    const long long ht = i / TPR;
+    const int h = static_cast<int>(ht / total_q);
+    const long long t = ht - static_cast<long long>(h) * total_q;
+    const float4 a = acc[2 * i], b = acc[2 * i + 1];
+    dq[(t * H + h) * TPR + part] =
+        make_uint4(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale),
+                   pack2<BF16>(b.x * scale, b.y * scale), pack2<BF16>(b.z * scale, b.w * scale));
 }
 
 // ---------------------------------------------------------------------------
@@ -248,7 +330,7 @@ struct BwdCfg {
 
 constexpr int kErrSmemAlign = 5;   // matches FA_ERR_CUDA
 
-template <int D, int NS, bool BF16, bool GENERAL>
+template <int D, int NS, bool BF16, bool GENERAL, bool VARLEN = false>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -256,6 +338,38 @@ __global__ void __launch_bounds__(512, 1)
                const BwdParams p) {
     using C = BwdCfg<D, NS>;
     constexpr int BM = C::BM;
+    static_assert(GENERAL || !VARLEN, "packed batches use the general band");
+    // one-dimensional grid, (batch, head) minor: causal runs the heaviest key
+    // blocks (j = 0) of every (b, h) first (longest work first)
+    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+    const int j = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    // packed variable-length batches: the grid is sized by the longest
+    // sequence; a CTA past its own sequence's keys leaves before any setup.
+    // lp is p with this sequence's lengths; TMA rows are offset by qrow0 /
+    // krow0 in plane (the head)
+    BwdParams lp;
+    int qrow0 = 0, krow0 = 0, plane = bh;
+    if constexpr (VARLEN) {
+        const int b = bh / p.H;
+        plane = bh - b * p.H;
+        const SeqSpan sq = seq_span(p.cu_q, b, p.total_q, p.Nq);
+        const SeqSpan sk = seq_span(p.cu_k, b, p.total_k, p.Nk);
+        if (j * 128 >= sk.len) return;
+        lp = p;
+        lp.Nq = sq.len;
+        lp.Nk = sk.len;
+        lp.nqt = (sq.len + BM - 1) / BM;
+        lp.nkb = (sk.len + 127) / 128;
+        lp.off = sk.len - sq.len;
+        qrow0 = sq.start;
+        krow0 = sk.start;
+    }
+    const BwdParams &ip = pick<VARLEN>(lp, p);
+    // accumulator row of this (b, h)'s query row q
+    auto dq_row = [&](int q) -> size_t {
+        if constexpr (VARLEN) return static_cast<size_t>(plane) * p.total_q + qrow0 + q;
+        else return static_cast<size_t>(bh) * p.Nq + q;
+    };
     extern __shared__ __align__(1024) uint8_t smem_buf[];
     if (smem_u32(smem_buf) & 1023u) {
         if (threadIdx.x == 0) atomicCAS(&g_dev_status, 0, kErrSmemAlign);
@@ -265,10 +379,6 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // one-dimensional grid, (batch, head) minor: causal runs the heaviest key
-    // blocks (j = 0) of every (b, h) first (longest work first)
-    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
-    const int j = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -318,14 +428,16 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVTile);
                 for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(sbase + C::kKOff + c * C::kChunk, &tmk, bar(C::kBarKV), c * 64, j * 128, bh);
-                    tma_load_3d(sbase + C::kVOff + c * C::kChunk, &tmv, bar(C::kBarKV), c * 64, j * 128, bh);
+                    tma_load_3d(sbase + C::kKOff + c * C::kChunk, &tmk, bar(C::kBarKV), c * 64, krow0 + j * 128,
+                                plane);
+                    tma_load_3d(sbase + C::kVOff + c * C::kChunk, &tmv, bar(C::kBarKV), c * 64, krow0 + j * 128,
+                                plane);
                 }
             }
             __syncwarp();
             QIter<BM, GENERAL> it;
             int i;
-            while (it.next(p, j, i)) {
+            while (it.next(ip, j, i)) {
                 const int s = cnt % NS;
                 // Q_i with the padded LSE_i, dO_i with D_i (TMA tiles and bulk
                 // copies of the statistics prepared by bwd_pre), each pair on
@@ -338,7 +450,8 @@ __global__ void __launch_bounds__(512, 1)
                     const uint32_t qb = bar(C::kBarQFull + s);
                     mbar_arrive_expect_tx(qb, C::kQTile + C::kStatBytes);
                     for (int c = 0; c < D / 64; ++c)
-                        tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kChunk, &tmq, qb, c * 64, i * BM, bh);
+                        tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kChunk, &tmq, qb, c * 64,
+                                    qrow0 + i * BM, plane);
                     bulk_load(st, p.lse2 + srow, C::kStatBytes, qb);
                 }
                 __syncwarp();
@@ -348,7 +461,8 @@ __global__ void __launch_bounds__(512, 1)
                     const uint32_t ob = bar(C::kBarOFull + s);
                     mbar_arrive_expect_tx(ob, C::kQTile + C::kStatBytes);
                     for (int c = 0; c < D / 64; ++c)
-                        tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kChunk, &tmdo, ob, c * 64, i * BM, bh);
+                        tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kChunk, &tmdo, ob, c * 64,
+                                    qrow0 + i * BM, plane);
                     bulk_load(st + C::kStatBytes, p.dvec + srow, C::kStatBytes, ob);
                 }
                 __syncwarp();
@@ -411,7 +525,7 @@ __global__ void __launch_bounds__(512, 1)
 
             QIter<BM, GENERAL> it;
             int i, in;
-            bool have = it.next(p, j, i);
+            bool have = it.next(ip, j, i);
             if (have) {
                 ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
                 if (ok) {
@@ -432,7 +546,7 @@ __global__ void __launch_bounds__(512, 1)
                 const int s = cnt % NS;
                 const int sn = (cnt + 1) % NS;
                 const uint32_t ph = cnt & 1;
-                const bool have_n = it.next(p, j, in);
+                const bool have_n = it.next(ip, j, in);
                 ok = wait_bar(bar(C::kBarPFull), ph, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -498,7 +612,7 @@ __global__ void __launch_bounds__(512, 1)
             const float c = p.scale_log2;
             QIter<BM, GENERAL> it;
             int i;
-            while (it.next(p, j, i)) {
+            while (it.next(ip, j, i)) {
                 const int s = cnt % NS;
                 const uint32_t ph = cnt & 1;
                 ok = wait_bar(bar(C::kBarSFull), ph, abort_flag) &&
@@ -516,10 +630,10 @@ __global__ void __launch_bounds__(512, 1)
                 int qk, lo, hi;
                 bool masked;
                 if constexpr (GENERAL) {
-                    qk = key - p.off - (i * BM + q0);     // |values| < 2^30 (Nq, Nk <= 2^28)
+                    qk = key - ip.off - (i * BM + q0);     // |values| < 2^30 (Nq, Nk <= 2^28)
                     lo = max(qk - p.wr, -1);
                     hi = min(qk + p.wl, 64);
-                    if (key >= p.Nk) lo = 64;
+                    if (key >= ip.Nk) lo = 64;
                     masked = __any_sync(0xffffffffu, lo > 0 || hi < 63);
                 } else {
                     // square: the diagonal tile hides queries before the key
@@ -617,6 +731,10 @@ __global__ void __launch_bounds__(512, 1)
                 // a key block that no query tile sees never waited for its K/V
                 // loads: they must land before the staging areas are written
                 if (done && cnt == 0) drain_bar(bar(C::kBarKV), 0);
+                // packed batches: a key block that ends inside the next
+                // sequence's rows is written row by row with plain stores (a
+                // TMA store clips only at the end of the tensor)
+                const int krows = VARLEN ? ip.Nk - j * 128 : 128;
                 if (done) {
         #pragma unroll 1
                     for (int ch = 0; ch < D / 32; ++ch) {
@@ -631,6 +749,17 @@ __global__ void __launch_bounds__(512, 1)
     #pragma unroll
                         for (int k = 0; k < 16; ++k)
                             pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+                        if (VARLEN && krows < 128) {
+                            if (r < krows) {
+                                uint4 *g = reinterpret_cast<uint4 *>(
+                                    static_cast<uint8_t *>(is_dv ? p.dv : p.dk) +
+                                    (static_cast<size_t>(krow0 + j * 128 + r) * p.H + plane) * (D * 2) + ch * 64);
+    #pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    g[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                            }
+                            continue;
+                        }
                         uint8_t *srow = stage + (ch >> 1) * C::kChunk + r * 128;
     #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -642,9 +771,10 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 fence_async_smem();
                 named_sync(is_dv ? 1 : 2, 128);   // the four warps of this output (every one gets here)
-                if (done && (warp & 3) == 0 && lane == 0) {
+                if (done && krows >= 128 && (warp & 3) == 0 && lane == 0) {
                     for (int c = 0; c < D / 64; ++c)   // keys >= Nk are clipped
-                        tma_store_3d(is_dv ? &tmdv : &tmdk, smem_u32(stage + c * C::kChunk), c * 64, j * 128, bh);
+                        tma_store_3d(is_dv ? &tmdv : &tmdk, smem_u32(stage + c * C::kChunk), c * 64,
+                                     krow0 + j * 128, plane);
                     bulk_commit();
                     bulk_wait_read();
                 }
@@ -661,7 +791,7 @@ __global__ void __launch_bounds__(512, 1)
             int nh = 0;                                  // d = 64: staged halves
             QIter<BM, GENERAL> it;
             int i;
-            while (p.dqacc != nullptr && it.next(p, j, i)) {
+            while (p.dqacc != nullptr && it.next(ip, j, i)) {
                 ok = wait_bar(bar(C::kBarDqFull), cnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -684,7 +814,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int q0 = i * BM + 64 * h;
-                        const int rows = min(64, p.Nq - q0);
+                        const int rows = min(64, ip.Nq - q0);
                         if (rows <= 0) break;
                         // staging half h was last read by the reduction two before
                         if (issuer) {
@@ -704,7 +834,7 @@ __global__ void __launch_bounds__(512, 1)
                             ok = wait_bar(bar(C::kBarDqStaged), nh & 1, abort_flag);
                             if (!ok) break;
                             if (issuer) {
-                                bulk_reduce_add_f32(p.dqacc + (static_cast<size_t>(bh) * p.Nq + q0) * D,
+                                bulk_reduce_add_f32(p.dqacc + dq_row(q0) * D,
                                                     sbase + C::kDqStageOff + h * C::kDqHalf,
                                                     static_cast<uint32_t>(rows) * D * 4);
                                 bulk_commit();
@@ -714,8 +844,8 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (!ok) break;
                 } else if (row_lane) {
-                    float *acc = p.dqacc + (static_cast<size_t>(bh) * p.Nq + static_cast<size_t>(i) * BM) * D + dcol;
-                    const int lim = p.Nq - i * BM;
+                    float *acc = p.dqacc + dq_row(i * BM) * D + dcol;
+                    const int lim = ip.Nq - i * BM;
 #pragma unroll
                     for (int k = 0; k < BM; ++k)
                         if (k < lim) atomicAdd(acc + k * D, __uint_as_float(v[k]));

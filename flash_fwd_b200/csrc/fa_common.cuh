@@ -58,6 +58,35 @@ __device__ __forceinline__ bool band_any(int q0, int q1, int k0, int k1, int off
 }
 
 // ---------------------------------------------------------------------------
+// Packed variable-length batches: sequence b owns the packed rows
+// cu[b] .. cu[b+1]-1 (cu: DEVICE int32 [B + 1], cumulative lengths).  The
+// bounds are clamped into [0, total] and the length to max_len, so that no
+// access leaves the caller's buffers whatever cu holds; a clamp that changed
+// anything records kErrInvalid in the device status word.
+// ---------------------------------------------------------------------------
+constexpr int kErrInvalid = 1;           // matches FA_ERR_INVALID_ARG
+
+// a when V, else b (the per-sequence parameters of a packed batch, or the
+// kernel's own)
+template <bool V, typename T>
+__device__ __forceinline__ const T &pick(const T &a, const T &b) {
+    if constexpr (V) return a;
+    else return b;
+}
+
+struct SeqSpan {
+    int start, len;
+};
+
+__device__ __forceinline__ SeqSpan seq_span(const int *cu, int b, int total, int max_len) {
+    const int a = __ldg(cu + b), e = __ldg(cu + b + 1);
+    const int s = min(max(a, 0), total);
+    const int t = min(max(e, s), total);
+    if (a < 0 || e < a || e > total || t - s > max_len) atomicCAS(&g_dev_status, 0, kErrInvalid);
+    return SeqSpan{s, min(t - s, max_len)};
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -64,6 +64,14 @@ struct FwdParams {
     int mode;                 // kCausal (heaviest-first order) | kSparse bits
     float scale;
     float scale_log2;         // scale * log2(e)
+    // packed variable-length batches (VARLEN kernels): sequence b owns packed
+    // rows cu_q[b] .. cu_q[b+1]-1 of q and o and cu_k[b] .. cu_k[b+1]-1 of k
+    // and v, each [rows][H][d]; lse is [H][total_q].  Nq, Nk, nqb and nkb
+    // above then describe the longest sequences (they size the item grid).
+    const int *cu_q;
+    const int *cu_k;
+    void *o;                  // packed O: the rows of a sequence's last, partial tile
+    int total_q, total_k;     // packed rows
 };
 
 // Is key block j visible at all from query block rb?  GENERAL kernels handle
@@ -188,6 +196,58 @@ __device__ __forceinline__ void fwd_decode(const FwdParams &p, int item, int &bh
     rb0 = ((p.mode & kCausal) ? nqp - 1 - qi : qi) * NQ;
 }
 
+// The items a CTA runs, in turn r = 0, 1, ...  Dense problems: item
+// fwd_item(r) of the grid above.  Packed variable-length batches (VARLEN):
+// the same grid, sized by the longest sequence, walked in the same order with
+// the positions past a sequence's own query groups skipped (v counts the
+// positions walked); lp is then p with the item's sequence lengths, and the
+// TMA coordinates of its rows are offset by qrow0 / krow0 in plane h.  Every
+// role of the CTA walks the same items.
+template <int NQ, bool VARLEN>
+struct FwdWalk {
+    int v = 0;
+    int bh = 0, rb0 = 0;
+    int qrow0 = 0, krow0 = 0, plane = 0;
+    FwdParams lp;
+    __device__ __forceinline__ const FwdParams &prm(const FwdParams &p) const {
+        if constexpr (VARLEN) return lp;
+        else return p;
+    }
+    __device__ __forceinline__ bool next(const FwdParams &p, int r, int cta, int G) {
+        if constexpr (!VARLEN) {
+            const int item = fwd_item(r, cta, G);
+            if (item >= p.nitems) return false;
+            fwd_decode<NQ>(p, item, bh, rb0);
+            plane = bh;
+            return true;
+        } else {
+            for (;;) {
+                const int item = fwd_item(v++, cta, G);
+                if (item >= p.nitems) return false;
+                bh = item % p.nbh;
+                const int qi = item / p.nbh;
+                const int b = bh / p.H;
+                plane = bh - b * p.H;
+                const SeqSpan sq = seq_span(p.cu_q, b, p.total_q, p.Nq);
+                const int nqb = (sq.len + 127) / 128;
+                const int nqp = (nqb + NQ - 1) / NQ;
+                if (qi >= nqp) continue;
+                const SeqSpan sk = seq_span(p.cu_k, b, p.total_k, p.Nk);
+                rb0 = ((p.mode & kCausal) ? nqp - 1 - qi : qi) * NQ;
+                lp = p;
+                lp.Nq = sq.len;
+                lp.Nk = sk.len;
+                lp.nqb = nqb;
+                lp.nkb = (sk.len + 127) / 128;
+                lp.off = sk.len - sq.len;
+                qrow0 = sq.start;
+                krow0 = sk.start;
+                return true;
+            }
+        }
+    }
+};
+
 // A CTA stays resident and runs its work items in turn.  Within an item the
 // roles work as described at the top of this file; across items:
 //   - the K producer loads the next item's Q once every S product of the
@@ -199,12 +259,13 @@ __device__ __forceinline__ void fwd_decode(const FwdParams &p, int item, int &bh
 //   - the MMA warp completes OFull_t of an item only after the epilogue of the
 //     item before has read O_t from TMEM (OFree_t), so each of these barriers
 //     completes once per item, in step with its waiter.
-template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL>
+template <int D, int NQ, int NSK, int NSV, bool BF16, bool GENERAL, bool VARLEN = false>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, const FwdParams p) {
     using C = FwdCfg<D, NQ, NSK, NSV>;
     static_assert(NSV >= NQ, "O_t is staged in V stage t");
+    static_assert(GENERAL || !VARLEN, "packed batches use the general band");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -266,14 +327,36 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             // TMA stores of item r's O tiles from V stages 0 .. NQ-1, once the
             // softmax warps have staged them; the stages are reloaded only
             // after the stores have read them
-            auto store_item = [&](int r, int bh, int rb0) -> bool {
+            auto store_item = [&](int r, int bh, int rb0, int nqb, int nq, int qrow0) -> bool {
                 const bool ok = wait_bar(bar(C::kBarOStaged), r & 1, abort_flag);
-                if (ok && lane == 0) {
+                if (!ok) return ok;
+                if constexpr (VARLEN) {
+                    // a tile that ends inside the packed rows of the next
+                    // sequence is written row by row with plain stores (a TMA
+                    // store clips only at the end of the tensor)
                     for (int t = 0; t < NQ; ++t) {
-                        if (rb0 + t >= p.nqb) continue;
+                        const int rows = nq - (rb0 + t) * 128;
+                        if (rb0 + t >= nqb || rows >= 128) continue;
+                        const uint8_t *stage = smem + C::kVOff + t * C::kTileBytes;
+                        uint8_t *dst = static_cast<uint8_t *>(p.o) +
+                                       (static_cast<size_t>(qrow0 + (rb0 + t) * 128) * p.H + bh % p.H) * (D * 2);
+                        for (int e = lane; e < rows * C::kChunks * 8; e += 32) {
+                            const int rr = e / (C::kChunks * 8), c = (e >> 3) % C::kChunks, u = e & 7;
+                            *reinterpret_cast<uint4 *>(dst + static_cast<size_t>(rr) * p.H * (D * 2) + c * 128 +
+                                                       u * 16) =
+                                *reinterpret_cast<const uint4 *>(stage + c * C::kChunkBytes + rr * 128 +
+                                                                 ((u ^ (rr & 7)) << 4));
+                        }
+                    }
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    for (int t = 0; t < NQ; ++t) {
+                        if (rb0 + t >= nqb) continue;
+                        if (VARLEN && nq - (rb0 + t) * 128 < 128) continue;
                         for (int c = 0; c < C::kChunks; ++c)   // rows >= Nq are clipped
                             tma_store_3d(&tmo, sbase + C::kVOff + t * C::kTileBytes + c * C::kChunkBytes, c * 64,
-                                         (rb0 + t) * 128, bh);
+                                         qrow0 + (rb0 + t) * 128, VARLEN ? bh % p.H : bh);
                     }
                     bulk_commit();
                     bulk_wait_read();
@@ -284,15 +367,15 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             };
             int nk = 0, nv = 0;   // loads issued (all items)
             int nit = 0;          // items started
-            int pbh = 0, prb0 = 0;
+            int pbh = 0, prb0 = 0, pnqb = 0, pnq = 0, pq0 = 0;
             bool ok = true;
+            FwdWalk<NQ, VARLEN> w;
             for (int r = 0; ok; ++r) {
-                const int item = fwd_item(r, cta, G);
-                if (item >= p.nitems) break;
-                int bh, rb0;
-                fwd_decode<NQ>(p, item, bh, rb0);
+                if (!w.next(p, r, cta, G)) break;
+                const FwdParams &ip = w.prm(p);
+                const int bh = w.bh, rb0 = w.rb0;
                 if (do_v && r > 0) {
-                    ok = store_item(r - 1, pbh, prb0);
+                    ok = store_item(r - 1, pbh, prb0, pnqb, pnq, pq0);
                     if (!ok) break;
                 }
                 if (do_k) {
@@ -302,13 +385,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     }
                     if (lane == 0) {
                         int nq_valid = 0;
-                        for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < p.nqb) ? 1 : 0;
+                        for (int t = 0; t < NQ; ++t) nq_valid += (rb0 + t < ip.nqb) ? 1 : 0;
                         mbar_arrive_expect_tx(bar(C::kBarQ), nq_valid * C::kTileBytes);
                         for (int t = 0; t < NQ; ++t) {
-                            if (rb0 + t >= p.nqb) continue;
+                            if (rb0 + t >= ip.nqb) continue;
                             for (int c = 0; c < C::kChunks; ++c)
                                 tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + c * C::kChunkBytes, &tmq,
-                                            bar(C::kBarQ), c * 64, (rb0 + t) * 128, bh);
+                                            bar(C::kBarQ), c * 64, w.qrow0 + (rb0 + t) * 128, w.plane);
                         }
                     }
                     __syncwarp();
@@ -317,7 +400,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 KvIter<NQ, GENERAL> it;
                 int j;
                 uint32_t f;
-                while (ok && it.next(p, rb0, j, f)) {
+                while (ok && it.next(ip, rb0, j, f)) {
                     if (do_k) {
                         const int s = nk % NSK;
                         ok = wait_bar(bar(C::kBarKEmpty + s), ((nk / NSK) & 1) ^ 1u, abort_flag);
@@ -326,7 +409,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                             mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
                             for (int c = 0; c < C::kChunks; ++c)
                                 tma_load_3d(sbase + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, &tmk,
-                                            bar(C::kBarKFull + s), c * 64, j * 128, bh);
+                                            bar(C::kBarKFull + s), c * 64, w.krow0 + j * 128, w.plane);
                         }
                         ++nk;
                     }
@@ -338,7 +421,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                             mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
                             for (int c = 0; c < C::kChunks; ++c)
                                 tma_load_3d(sbase + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, &tmv,
-                                            bar(C::kBarVFull + s), c * 64, j * 128, bh);
+                                            bar(C::kBarVFull + s), c * 64, w.krow0 + j * 128, w.plane);
                         }
                         ++nv;
                     }
@@ -346,9 +429,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 }
                 pbh = bh;
                 prb0 = rb0;
+                pnqb = ip.nqb;
+                pnq = ip.Nq;
+                pq0 = w.qrow0;
             }
             // the last item's outputs
-            if (do_v && ok && nit > 0) store_item(nit - 1, pbh, prb0);
+            if (do_v && ok && nit > 0) store_item(nit - 1, pbh, prb0, pnqb, pnq, pq0);
             // every issued load has landed before the CTA may exit
             if (do_k && nit > 0) drain_bar(bar(C::kBarQ), (nit - 1) & 1);
             for (int i = (nk > NSK ? nk - NSK : 0); i < nk; ++i)
@@ -387,19 +473,18 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
 #pragma unroll
             for (int t = 0; t < NQ; ++t) pc[t] = 0;
             bool ok = true;
+            FwdWalk<NQ, VARLEN> w;
             for (int r = 0; ok; ++r) {
-                const int item = fwd_item(r, cta, G);
-                if (item >= p.nitems) break;
-                int bh, rb0;
-                fwd_decode<NQ>(p, item, bh, rb0);
-                (void)bh;
+                if (!w.next(p, r, cta, G)) break;
+                const FwdParams &ip = w.prm(p);
+                const int rb0 = w.rb0;
                 int ci[NQ];    // P_t V products of this item (accumulate after the first)
 #pragma unroll
                 for (int t = 0; t < NQ; ++t) ci[t] = 0;
                 KvIter<NQ, GENERAL> it;
                 int j, jn;
                 uint32_t f, fn;
-                bool have = it.next(p, rb0, j, f);
+                bool have = it.next(ip, rb0, j, f);
                 ok = wait_bar(bar(C::kBarQ), r & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -427,7 +512,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     const int ki = kc + u + 1;             // K tile of the next key tile
                     const int sn = ki % NSK;
                     const uint32_t phn = (ki / NSK) & 1;
-                    const bool have_n = it.next(p, rb0, jn, fn);
+                    const bool have_n = it.next(ip, rb0, jn, fn);
                     if (!have_n) {
                         // every S product of the item is issued: Q may be replaced
                         mma_commit(bar(C::kBarQEmpty), leader);
@@ -504,11 +589,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
         const float c = p.scale_log2;
         int sc = 0;            // S_t products consumed, all items (parity of SFull_t)
         bool ok = true;
+        FwdWalk<NQ, VARLEN> w;
         for (int ri = 0; ok; ++ri) {
-            const int item = fwd_item(ri, cta, G);
-            if (item >= p.nitems) break;
-            int bh, rb0;
-            fwd_decode<NQ>(p, item, bh, rb0);
+            if (!w.next(p, ri, cta, G)) break;
+            const FwdParams &ip = w.prm(p);
+            const int bh = w.bh, rb0 = w.rb0;
             const int rb = rb0 + t;
             const int row = rb * 128 + row_local;
             float m = -INFINITY, l = 0.f, l_r = 0.f;
@@ -521,7 +606,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
             KvIter<NQ, GENERAL> it;
             int j;
             uint32_t f;
-            while (it.next(p, rb0, j, f)) {
+            while (it.next(ip, rb0, j, f)) {
                 if (!((f >> t) & 1u)) continue;
                 ok = wait_bar(bar(C::kBarSFull + t), sc & 1, abort_flag);
                 if (!ok) break;
@@ -542,9 +627,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 // this row's visible keys within the tile: [lo, hi]
                 int lo, hi, rk = 0;
                 if constexpr (GENERAL) {
-                    rk = row + p.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
+                    rk = row + ip.off - j * 128;     // |values| < 2^30 (Nq, Nk <= 2^28)
                     lo = max(rk - p.wl, -1);
-                    hi = min(min(rk + p.wr, p.Nk - 1 - j * 128), 128);
+                    hi = min(min(rk + p.wr, ip.Nk - 1 - j * 128), 128);
                 } else {
                     lo = -1;
                     hi = 127;
@@ -661,7 +746,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 ok = wait_bar(bar(C::kBarStoreRead), (ri - 1) & 1, abort_flag);
                 if (!ok) break;
             }
-            if (rb < p.nqb) {
+            if (rb < ip.nqb) {
                 uint8_t *stage = smem + C::kVOff + t * C::kTileBytes;
                 const float l_o = BF16 ? l_r : l;
                 // a row that saw no key: O = 0, LSE = -inf
@@ -688,9 +773,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                             make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
                     }
                 }
-                if (row < p.Nq) {
+                if (row < ip.Nq) {
                     const float lse = (seen && l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                    p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
+                    if constexpr (VARLEN)
+                        p.lse[static_cast<size_t>(w.plane) * p.total_q + w.qrow0 + row] = lse;
+                    else
+                        p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse;
                 }
             }
             tc_fence_before();

@@ -90,6 +90,31 @@ def make_qkv_cross(B, H, Nq, Nk, d, dtype="bf16", seed=0, qk_std=1.0):
     return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous(), do.to(t).contiguous()
 
 
+def make_varlen(lengths_q, lengths_k, H, d, dtype="bf16", seed=0):
+    """A packed batch: cu_seqlens_q, cu_seqlens_k (int32 [B + 1]), Q, dO
+    [total_q, H, d] and K, V [total_k, H, d] CPU tensors of ``dtype`` (draw
+    order Q, K, V, dO, as in make_qkv)."""
+    lq = torch.tensor([0] + list(lengths_q), dtype=torch.int64)
+    lk = torch.tensor([0] + list(lengths_k), dtype=torch.int64)
+    assert len(lq) == len(lk) and bool((lq >= 0).all()) and bool((lk >= 0).all())
+    cu_q, cu_k = torch.cumsum(lq, 0).to(torch.int32), torch.cumsum(lk, 0).to(torch.int32)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn((tq, H, d), generator=g, dtype=torch.float32)
+    k = torch.randn((tk, H, d), generator=g, dtype=torch.float32)
+    v = torch.randn((tk, H, d), generator=g, dtype=torch.float32)
+    do = torch.randn((tq, H, d), generator=g, dtype=torch.float32)
+    t = DTYPES[dtype]
+    return cu_q, cu_k, q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous(), do.to(t).contiguous()
+
+
+def varlen_lengths(B, lo, hi, seed=0):
+    """B sequence lengths drawn uniformly from [lo, hi] (seeded): the length mix
+    of a packed batch."""
+    g = torch.Generator().manual_seed(int(seed) + 104729)
+    return [int(x) for x in torch.randint(lo, hi + 1, (B,), generator=g)]
+
+
 def alibi_slopes(H):
     """The geometric head slopes 2^(-8 (h + 1) / H) commonly used with ALiBi (fp32 [H])."""
     return torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32)

@@ -156,6 +156,54 @@ FA_API int fa_bwd_ex(const void *q, const void *k, const void *v, const void *o,
                      const uint8_t *block_mask, int dtype, void *stream);
 
 /*
+ * Packed variable-length batches (the varlen form of the flash_attn_func
+ * interface of "FlashAttention原理概览" section 3.4): B sequences of
+ * different lengths concatenated along the token axis, each attending only
+ * within itself.
+ *   q, o      [total_q][H][d]   k, v [total_k][H][d]   (token major, d innermost)
+ *   lse       fp32 [H][total_q]
+ *   cu_seqlens_q, cu_seqlens_k   DEVICE int32 [B + 1], 4-byte aligned: the
+ *             cumulative lengths; sequence b owns query rows
+ *             cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key rows
+ *             cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.  They should start at
+ *             0, never decrease and end at total_q / total_k; sequences may
+ *             be empty.
+ *   max_seqlen_q, max_seqlen_k   host upper bounds of the lengths (they size
+ *             the grids), 1 <= max_seqlen <= total.
+ * Within sequence b the problem is the one of fa_fwd_ex with Nq, Nk its own
+ * lengths: causal and window are bottom-right aligned per sequence, and
+ * alibi_slopes are per head.  Query rows of a sequence with no keys get
+ * O = 0, LSE = -inf.  Block masks are not accepted (FA_ERR_UNSUPPORTED).
+ * The library cannot read cu_seqlens on the host: the kernels clamp every
+ * bound into [0, total] and every length to max_seqlen, so that nothing
+ * outside the buffers is touched whatever the arrays hold, and record
+ * FA_ERR_INVALID_ARG for fa_last_device_status() when a clamp changed
+ * anything (the outputs are then incomplete).
+ */
+FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                         const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                         int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal, int window_left,
+                         int window_right, const float *alibi_slopes, int dtype, void *stream);
+
+/*
+ * Workspace of fa_bwd_varlen: the two fp32 statistics [B][H][Npad] (Npad =
+ * max_seqlen_q rounded up to FA_BLOCK) and the fp32 dQ accumulator
+ * [H][total_q][d].  0 for invalid sizes (d = 256 included).
+ */
+FA_API size_t fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d);
+
+/*
+ * Backward of fa_fwd_varlen with the same arguments: dq [total_q][H][d],
+ * dk, dv [total_k][H][d].  d = 64 or 128 (256: FA_ERR_UNSUPPORTED); dq is
+ * accumulated with fp32 atomics as in fa_bwd.
+ */
+FA_API int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                         const float *lse, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                         const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                         int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal, int window_left,
+                         int window_right, const float *alibi_slopes, int dtype, void *stream);
+
+/*
  * Bytes of device workspace fa_bwd_deterministic needs: the two fp32 per-row
  * statistics [B][H][Npad] only (no dQ accumulator).  0 for invalid sizes.
  */

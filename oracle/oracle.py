@@ -217,6 +217,69 @@ def bwd_dkdv_cols(q, k, v, dout, scale, cols, flags=0, mask=None, blk=128, nthre
 
 
 # --------------------------------------------------------------------------
+# Packed variable-length batches.  Sequence b is an attention problem of its
+# own: query rows cu_q[b] .. cu_q[b+1]-1 against key rows cu_k[b] ..
+# cu_k[b+1]-1 (bottom-right aligned as above), so the packed result is the
+# per-sequence definition applied to each slice ("FlashAttention原理概览"
+# section 3.4 interface, its variable-length form).  Packed tensors are
+# [total, H, d]; LSE is [H, total_q].  A row whose sequence has no keys gets
+# O = 0, LSE = -inf and zero gradients.
+# --------------------------------------------------------------------------
+def _bounds(cu):
+    cu = np.asarray(cu, dtype=np.int64).reshape(-1)
+    assert cu.ndim == 1 and len(cu) >= 2 and cu[0] == 0 and np.all(np.diff(cu) >= 0), "cumulative lengths"
+    return cu
+
+
+def _heads(x):
+    """[n, H, d] packed slice -> [H, n, d]."""
+    return np.ascontiguousarray(np.transpose(_f64(x), (1, 0, 2)))
+
+
+def fwd_varlen(q, k, v, cu_q, cu_k, scale, flags=0, window=None, slopes=None, nthreads=None):
+    """O [total_q, H, d] and LSE [H, total_q] of a packed batch."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq, ck = _bounds(cu_q), _bounds(cu_k)
+    assert len(cq) == len(ck) and cq[-1] == q.shape[0] and ck[-1] == k.shape[0]
+    total_q, H, d = q.shape
+    o = np.zeros((total_q, H, d))
+    lse = np.full((H, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        ob, lb = fwd(_heads(q[q0:q1]), _heads(k[k0:k1]), _heads(v[k0:k1]), scale, flags, nthreads=nthreads,
+                     window=window, slopes=slopes)
+        o[q0:q1] = np.transpose(ob, (1, 0, 2))
+        lse[:, q0:q1] = lb
+    return o, lse
+
+
+def bwd_varlen(q, k, v, dout, cu_q, cu_k, scale, flags=0, window=None, slopes=None, nthreads=None):
+    """(O, LSE, dQ, dK, dV) of a packed batch, each sequence by bwd_full."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cq, ck = _bounds(cu_q), _bounds(cu_k)
+    assert len(cq) == len(ck) and cq[-1] == q.shape[0] and ck[-1] == k.shape[0]
+    total_q, H, d = q.shape
+    o, dq = np.zeros_like(q), np.zeros_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(k)
+    lse = np.full((H, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        ob, lb, dqb, dkb, dvb = bwd_full(_heads(q[q0:q1]), _heads(k[k0:k1]), _heads(v[k0:k1]),
+                                         _heads(dout[q0:q1]), scale, flags, nthreads=nthreads, window=window,
+                                         slopes=slopes)
+        o[q0:q1] = np.transpose(ob, (1, 0, 2))
+        lse[:, q0:q1] = lb
+        dq[q0:q1] = np.transpose(dqb, (1, 0, 2))
+        dk[k0:k1] = np.transpose(dkb, (1, 0, 2))
+        dv[k0:k1] = np.transpose(dvb, (1, 0, 2))
+    return o, lse, dq, dk, dv
+
+
+# --------------------------------------------------------------------------
 # FP8 forward (block quantisation + incoherent processing); the readings are
 # written out above the FP8 section of oracle.c
 # --------------------------------------------------------------------------
