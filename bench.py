@@ -88,7 +88,8 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    # 200 steps of the default workload time about 0.25 s: several clock samples
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsweep128", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -186,14 +187,23 @@ class ClockSampler:
         self.tmp = None
 
     def start(self):
+        """Starts sampling every 50 ms and returns once the first sample is in
+        (at most 3 s), so that the samples fall inside the region timed next."""
         try:
             self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
-            time.sleep(0.15)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t0 = time.monotonic()
+        while time.monotonic() - t0 < 3.0 and self.proc.poll() is None:
+            if os.path.getsize(self.tmp.name) > 0:
+                break
+            time.sleep(0.01)
+        # the first line may have been taken while the GPU idled: not a sample of the region
+        self.skip = 1 if os.path.getsize(self.tmp.name) > 0 else 0
 
     def stop(self):
         if self.proc is None:
@@ -207,7 +217,7 @@ class ClockSampler:
         with open(self.tmp.name) as f:
             lines = [ln.strip() for ln in f if ln.strip()]
         os.unlink(self.tmp.name)
-        return parse_clock_samples(lines)
+        return parse_clock_samples(lines[getattr(self, "skip", 0):])
 
 
 def parse_clock_samples(lines):
