@@ -88,8 +88,10 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # 200 steps of the default workload time about 0.25 s: several clock samples
-    ap.add_argument("--steps", type=int, default=200)
+    # 100 steps of the default workload time about 0.12 s, long enough for
+    # clock samples inside the region and short enough to stay a burst
+    # measurement (seconds-long runs settle under the 1000 W power cap)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsweep128", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -522,8 +522,8 @@ int launch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     {
-        // B x H x (key blocks of the longest sequence); CTAs past their own
-        // sequence's keys return at once
+        // B x (key blocks of the longest sequence) x H, sequence major; CTAs
+        // past their own sequence's keys return at once
         const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb));
         ProfScope prof(2, stream);
         kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, mdk, mdv, p);

@@ -224,6 +224,19 @@ __device__ __forceinline__ bool qtile_kept(const BwdParams &p, int i, int j) {
     return true;
 }
 
+// CTA blockIdx.x of a packed batch's backward grid, ordered sequence, key
+// block, head (nkb: key blocks of the longest sequence): its (sequence, head)
+// index b H + h and its key block.
+__device__ __forceinline__ int packed_bh(int nkb, int H) {
+    const unsigned per = static_cast<unsigned>(nkb) * static_cast<unsigned>(H);
+    const unsigned b = blockIdx.x / per;
+    return static_cast<int>(b * H + (blockIdx.x - b * per) % static_cast<unsigned>(H));
+}
+__device__ __forceinline__ int packed_j(int nkb, int H) {
+    const unsigned per = static_cast<unsigned>(nkb) * static_cast<unsigned>(H);
+    return static_cast<int>((blockIdx.x % per) / static_cast<unsigned>(H));
+}
+
 // Walks the query tiles that see key block j, in increasing order (warp-collective).
 template <int BM, bool GENERAL>
 struct QIter {
@@ -340,9 +353,12 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int BM = C::BM;
     static_assert(GENERAL || !VARLEN, "packed batches use the general band");
     // one-dimensional grid, (batch, head) minor: causal runs the heaviest key
-    // blocks (j = 0) of every (b, h) first (longest work first)
-    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
-    const int j = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    // blocks (j = 0) of every (b, h) first (longest work first).  Packed
+    // batches: sequence major, then key blocks, heads minor, so that the
+    // running CTAs reduce into the dQ rows of one or two sequences, which stay
+    // in L2 (in the (b, h)-minor order every sequence's rows are live at once)
+    const int bh = VARLEN ? packed_bh(p.nkb, p.H) : static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+    const int j = VARLEN ? packed_j(p.nkb, p.H) : static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
     // packed variable-length batches: the grid is sized by the longest
     // sequence; a CTA past its own sequence's keys leaves before any setup.
     // lp is p with this sequence's lengths; TMA rows are offset by qrow0 /
