@@ -32,6 +32,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -88,10 +89,11 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # 100 steps of the default workload time about 0.12 s, long enough for
-    # clock samples inside the region and short enough to stay a burst
-    # measurement (seconds-long runs settle under the 1000 W power cap)
-    ap.add_argument("--steps", type=int, default=100)
+    # the timed steps: a burst measurement (about 35 ms at the default
+    # workload); --sustained-steps then times a region long enough to settle
+    # under the 1000 W power cap, reported beside it
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--sustained-steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsweep128", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -178,19 +180,52 @@ def traffic_for(kernel, workload):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and throttle reasons sampled while the timed steps run.
+
+    NVML is read from a thread every 2 ms (so that even a region of a few tens
+    of milliseconds gets samples); where NVML is not available, nvidia-smi
+    samples every 50 ms.  Only reads: no clock or other setting is changed."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.tmp = None
+        self.nvml = None
+        self.thread = None
+        self.samples = []
 
     def start(self):
-        """Starts sampling every 50 ms and returns once the first sample is in
-        (at most 3 s), so that the samples fall inside the region timed next."""
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.running = True
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:   # no NVML here: nvidia-smi below
+            self.nvml = None
+        self._start_smi()
+
+    def _nvml_loop(self):
+        n = self.nvml
+        reason = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or n.nvmlDeviceGetCurrentClocksThrottleReasons
+        while self.running:
+            try:
+                self.samples.append((n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM), reason(self.handle)))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def _start_smi(self):
+        """Starts nvidia-smi every 50 ms and returns once its first sample is
+        in (at most 3 s), so that the samples fall inside the region timed next."""
         try:
             self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
@@ -208,6 +243,14 @@ class ClockSampler:
         self.skip = 1 if os.path.getsize(self.tmp.name) > 0 else 0
 
     def stop(self):
+        if self.nvml is not None:
+            self.running = False
+            self.thread.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            return summarise_nvml(self.samples, self.max_mhz)
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -219,7 +262,25 @@ class ClockSampler:
         with open(self.tmp.name) as f:
             lines = [ln.strip() for ln in f if ln.strip()]
         os.unlink(self.tmp.name)
-        return parse_clock_samples(lines[getattr(self, "skip", 0):])
+        out = parse_clock_samples(lines[getattr(self, "skip", 0):])
+        out["source"] = "nvidia-smi, 50 ms"
+        return out
+
+
+# NVML clock-event reason bits (nvml.h)
+NVML_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                0x80: "hw_power_brake_slowdown"}
+
+
+def summarise_nvml(samples, max_mhz):
+    """Median, minimum and maximum SM clock of NVML samples [(MHz, reason bits)]
+    and every reason seen active."""
+    reasons = sorted({name for _, bits in samples for bit, name in NVML_REASONS.items() if bits & bit})
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": reasons, "samples": 0, "source": "nvml, 2 ms"}
+    sm = [float(c) for c, _ in samples]
+    return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": float(max_mhz),
+            "reasons": reasons, "samples": len(sm), "source": "nvml, 2 ms"}
 
 
 def parse_clock_samples(lines):
@@ -615,6 +676,30 @@ def run_ours(args, w, name):
     # ---------------- dominant kernel roofline, per-kernel times, forward/backward split
     roof, kernel_times, split = analyse(prof, w, name, fwd_f, bwd_f, clocks, args.steps)
 
+    # ---------------- a sustained region: the same steps for about half a second or more
+    sustained = None
+    if args.sustained_steps > 0 and flush is None:
+        fdist.barrier(device)
+        torch.cuda.synchronize(device)
+        sampler = ClockSampler(local)
+        sampler.start()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.sustained_steps):
+            step(w, t, stream)
+        s1.record(stream)
+        torch.cuda.synchronize(device)
+        sclocks = sampler.stop()
+        sms = fdist.max_over_ranks(s0.elapsed_time(s1), device if args.gpus > 1 else None)
+        svalue = fdist.aggregate_throughput([flops * args.sustained_steps] * world, sms) / 1e12
+        _, ssus, _, psrc = peaks()
+        sustained = {"steps": args.sustained_steps, "ms_per_step": sms / args.sustained_steps, "value": svalue,
+                     "unit": UNIT, "clocks": sclocks, "sustained_peak": ssus,
+                     "peak_source": f"{psrc} bf16 sustained (MEASURED_PEAKS.json)"}
+        if fa.fa_last_device_status() != 0:
+            raise RuntimeError("device status after the sustained region is not ok")
+
     # ---------------- the same steps replayed from a CUDA graph (launch overhead removed)
     graph = None
     try:
@@ -701,6 +786,7 @@ def run_ours(args, w, name):
         "e2e": e2e,
         "clocks": clocks,
         "graph": graph,
+        "sustained": sustained,
         "device": device_info(local),
         "gpu_launches": sum(v[1] for v in prof.values()),
         "memory": memory,
