@@ -146,6 +146,28 @@ def test_clock_samples_are_summarised():
     assert bench.parse_clock_samples([])["sm_mhz"] is None
 
 
+def test_nvml_clock_samples_are_summarised():
+    # (SM MHz, NVML clock-event reason bits): 0x4 sw_power_cap, 0x8 hw_slowdown, 0x1 idle (ignored)
+    c = bench.summarise_nvml([(1965, 0x1), (1965, 0x4), (1500, 0x4), (1965, 0)], 1965)
+    assert c["samples"] == 4 and c["sm_mhz"] == 1965.0 and c["sm_min_mhz"] == 1500.0
+    assert c["reasons"] == ["sw_power_cap"] and bench.power_capped(c)
+    hot = bench.summarise_nvml([(1200, 0x8 | 0x40)], 1965)
+    assert hot["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    none = bench.summarise_nvml([], 1965)
+    assert none["sm_mhz"] is None and none["samples"] == 0
+
+
+def test_packed_workload_flops_sum_over_sequences():
+    from flash_fwd_b200 import accounting as acc
+    w = bench.WORKLOADS["varlen128"]
+    n = bench.varlen_lengths(w)
+    assert len(n) == w["B"] and all(w["varlen"][0] <= x <= w["varlen"][1] for x in n)
+    f, b = bench.workload_flops(w)
+    assert f == sum(acc.fwd_flops(1, w["H"], x, w["d"], True) for x in n) and b == 2.5 * f
+    per = [bench.head_flops(w, None, i) for i in range(w["B"] * w["H"])]
+    assert abs(sum(per) - (f + b)) <= 1e-6 * (f + b)
+
+
 def test_traffic_is_reported_only_for_unchanged_kernel_sources(tmp_path, monkeypatch):
     import json as _json
     sha = bench.kernel_source_sha()
