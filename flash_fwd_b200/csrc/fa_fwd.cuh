@@ -538,6 +538,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                             ++pc[t];
                             ++ci[t];
                         }
+                        // V_j is read by no later product: its stage is released when
+                        // the last P V completes, not after S of the next key tile too
+                        // (measured: +5.6 % at d = 256, where V has one stage; +0.3 to
+                        // +1.4 % at d = 128)
+                        if (t == NQ - 1) mma_commit(bar(C::kBarVEmpty + s), leader);
                         if (have_n && ((fn >> t) & 1u)) {
                             if (!k_ready) {
                                 ok = wait_bar(bar(C::kBarKFull + sn), phn, abort_flag);
@@ -551,7 +556,6 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                         }
                     }
                     if (!ok) break;
-                    mma_commit(bar(C::kBarVEmpty + s), leader);
                     if (have_n) mma_commit(bar(C::kBarKEmpty + sn), leader);
                     __syncwarp();
                     j = jn;

@@ -421,6 +421,9 @@ __global__ void __launch_bounds__(Fwd8Cfg<D>::kThreads, 1)
                         __syncwarp();
                         ++cnt[t];
                     }
+                    // V_j's stage is released when the last P V completes (as in the
+                    // 16-bit forward)
+                    if (t == NQ - 1) mma_commit(bar(C::kBarVEmpty + s), leader);
                     if ((fn >> t) & 1u) {
                         if (!k_ready) {
                             ok = wait_bar(bar(C::kBarKFull + sn), ((u + 1) / NSK) & 1, abort_flag);
@@ -434,7 +437,6 @@ __global__ void __launch_bounds__(Fwd8Cfg<D>::kThreads, 1)
                     }
                 }
                 if (!ok) break;
-                mma_commit(bar(C::kBarVEmpty + s), leader);
                 if (have_n) mma_commit(bar(C::kBarKEmpty + sn), leader);
                 __syncwarp();
             }
