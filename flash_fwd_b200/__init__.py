@@ -18,7 +18,7 @@ __all__ = [
     "fa_fwd_ex", "fa_bwd_ex", "fa_bwd_ex_workspace_bytes", "fa_bwd_deterministic",
     "fa_bwd_deterministic_workspace_bytes", "fa_fp8_quantize_qkv", "fa_fwd_fp8", "attention_fwd_fp8",
     "fa_bwd_noalloc", "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_bytes", "attention_fwd_varlen",
-    "attention_bwd_varlen",
+    "attention_bwd_varlen", "fa_bwd_varlen_deterministic", "fa_bwd_varlen_deterministic_workspace_bytes",
 ]
 
 FA_BLOCK = 128
@@ -69,6 +69,9 @@ def load_library():
     lib.fa_bwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_bwd_varlen_workspace_bytes.restype = sz
     lib.fa_bwd_varlen.argtypes = [vp] * 10 + [sz, vp, vp] + [i] * 7 + [f, i, i, i, vp, i, vp]
+    lib.fa_bwd_varlen_deterministic_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_varlen_deterministic_workspace_bytes.restype = sz
+    lib.fa_bwd_varlen_deterministic.argtypes = list(lib.fa_bwd_varlen.argtypes)
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_device_status.argtypes = []
@@ -78,7 +81,7 @@ def load_library():
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
                lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8, lib.fa_bwd_noalloc,
-               lib.fa_fwd_varlen, lib.fa_bwd_varlen,
+               lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_bwd_varlen_deterministic,
                lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
         fn.restype = ctypes.c_int
     _LIB = lib
@@ -452,17 +455,24 @@ def fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_q, d):
     return load_library().fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_q, d)
 
 
+def fa_bwd_varlen_deterministic_workspace_bytes(B, H, total_q, max_seqlen_q, d):
+    return load_library().fa_bwd_varlen_deterministic_workspace_bytes(B, H, total_q, max_seqlen_q, d)
+
+
 def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
-                  max_seqlen_k, causal=False, scale=None, window=None, alibi_slopes=None, stream=None):
+                  max_seqlen_k, causal=False, scale=None, window=None, alibi_slopes=None, stream=None,
+                  deterministic=False):
+    """Backward of a packed batch; deterministic=True: bitwise reproducible (fa_bwd_varlen_deterministic)."""
     B, H, tq, tk, d = _need_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dout,
                                    dq, dk, dv, workspace, alibi_slopes)
     wl, wr = _window(window)
-    rc = load_library().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+    lib = load_library()
+    rc = (lib.fa_bwd_varlen_deterministic if deterministic else lib.fa_bwd_varlen)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                       _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, tq, tk, int(max_seqlen_q),
                                       int(max_seqlen_k), d, _scale(scale, d), int(bool(causal)), wl, wr,
                                       _ptr(alibi_slopes), _dtype(q), _stream(stream))
-    _check(rc, "fa_bwd_varlen")
+    _check(rc, "fa_bwd_varlen_deterministic" if deterministic else "fa_bwd_varlen")
 
 
 def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False, scale=None,
@@ -476,13 +486,14 @@ def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_
 
 
 def attention_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                         causal=False, scale=None, window=None, alibi_slopes=None, workspace=None, stream=None):
+                         causal=False, scale=None, window=None, alibi_slopes=None, workspace=None, stream=None,
+                         deterministic=False):
     """Allocates dQ, dK, dV (and the workspace unless given) and runs the packed backward."""
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
-        nbytes = fa_bwd_varlen_workspace_bytes(cu_seqlens_q.numel() - 1, int(q.shape[1]), int(q.shape[0]),
-                                               int(max_seqlen_q), int(q.shape[2]))
+        ws = fa_bwd_varlen_deterministic_workspace_bytes if deterministic else fa_bwd_varlen_workspace_bytes
+        nbytes = ws(cu_seqlens_q.numel() - 1, int(q.shape[1]), int(q.shape[0]), int(max_seqlen_q), int(q.shape[2]))
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
-                  max_seqlen_k, causal, scale, window, alibi_slopes, stream)
+                  max_seqlen_k, causal, scale, window, alibi_slopes, stream, deterministic)
     return dq, dk, dv

@@ -458,26 +458,28 @@ int bwd_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, vo
 
 // ---------------------------------------------------------------- packed batches
 // Workspace of the packed backward: lse2 and D [BH][Npad] (Npad = the longest
-// query sequence rounded up to 128), then the fp32 dQ accumulator
-// [H][total_q][d].
-size_t bwd_varlen_workspace_bytes(long long BH, int H, int total_q, int max_nq, int d) {
+// query sequence rounded up to 128), then (not in the deterministic form) the
+// fp32 dQ accumulator [H][total_q][d].
+size_t bwd_varlen_workspace_bytes(long long BH, int H, int total_q, int max_nq, int d, bool deterministic) {
     return 2 * static_cast<size_t>(BH) * fa::bwd_npad(max_nq) * 4 +
-           static_cast<size_t>(H) * static_cast<size_t>(total_q) * d * 4;
+           (deterministic ? 0 : static_cast<size_t>(H) * static_cast<size_t>(total_q) * d * 4);
 }
 
-template <int D, bool BF16>
-int launch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk, cudaStream_t stream) {
-    using C = fa::BwdCfg<D, D == 64 ? 3 : 2>;
-    constexpr int BM = C::BM;
+// The packed backward: pre-pass, key-block kernel (bwd_kernel at d <= 128,
+// bwd_split_kernel at d = 256; BM-row query tiles), then the post-pass -- or,
+// deterministic, the key-block kernel without dQ and the dQ pass.
+template <int D, int BM, bool BF16, typename Kernel>
+int launch_bwd_varlen(Kernel kern, int smem_bytes, int threads, int split, const BwdBuffers &bb, const Problem &pr,
+                      const Packed &pk, bool deterministic, cudaStream_t stream) {
     const int BH = static_cast<int>(pr.BH());
     const int Npad = fa::bwd_npad(pr.Nq);
     float *lse2 = static_cast<float *>(bb.workspace);
     float *dvec = lse2 + static_cast<size_t>(BH) * Npad;
-    float *dqacc = dvec + static_cast<size_t>(BH) * Npad;
+    float *dqacc = deterministic ? nullptr : dvec + static_cast<size_t>(BH) * Npad;
     {
         constexpr int TPR = D / 8;
-        const long long threads = static_cast<long long>(BH) * Npad * TPR;
-        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        const long long nthreads = static_cast<long long>(BH) * Npad * TPR;
+        const unsigned blocks = static_cast<unsigned>((nthreads + 255) / 256);
         ProfScope prof(1, stream);
         fa::bwd_pre_varlen_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
             static_cast<const uint4 *>(bb.o), static_cast<const uint4 *>(bb.dout), bb.lse, lse2, dvec,
@@ -518,16 +520,32 @@ int launch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk,
     p.cu_k = pk.cu_k;
     p.total_q = pk.total_q;
     p.total_k = pk.total_k;
-    auto kern = fa::bwd_kernel<D, D == 64 ? 3 : 2, BF16, true, true>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
         return FA_ERR_CUDA;
     {
-        // B x (key blocks of the longest sequence) x H, sequence major; CTAs
-        // past their own sequence's keys return at once
-        const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb));
+        // B x (key blocks of the longest sequence) x H (x split), sequence
+        // major; CTAs past their own sequence's keys return at once
+        const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nkb * split));
         ProfScope prof(2, stream);
-        kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, mq, mdo, mdk, mdv, p);
+        kern<<<grid, threads, smem_bytes, stream>>>(mk, mv, mq, mdo, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if (deterministic) {
+        using C = fa::DqCfg<D>;
+        CUtensorMap mq1, mdo1, mdq;
+        if ((rc = make_map_packed(&mq1, bb.q, D, pk.total_q, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+        if ((rc = make_map_packed(&mdo1, bb.dout, D, pk.total_q, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+        if ((rc = make_map_packed(&mdq, bb.dq, D, pk.total_q, pr.H, pr.dtype, 128)) != FA_OK) return rc;
+        p.nqt = (pr.Nq + 127) / 128;
+        p.dq = bb.dq;
+        auto dkern = fa::bwd_dq_kernel<D, BF16, true, true>;
+        if (cudaFuncSetAttribute(dkern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+            return FA_ERR_CUDA;
+        // B x (query tiles of the longest sequence) x H, sequence major
+        const dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.nqt));
+        ProfScope prof(4, stream);
+        dkern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq1, mk, mv, mdo1, mdq, p);
+        return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
     }
     {
         const long long n8 = static_cast<long long>(pr.H) * pk.total_q * (D / 8);
@@ -540,26 +558,47 @@ int launch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk,
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <bool BF16>
+int dispatch_bwd_varlen(const BwdBuffers &bb, const Problem &pr, const Packed &pk, bool det, cudaStream_t s) {
+    switch (pr.d) {
+        case 64: {
+            using C = fa::BwdCfg<64, 3>;
+            return launch_bwd_varlen<64, 128, BF16>(fa::bwd_kernel<64, 3, BF16, true, true>, C::kSmemBytes,
+                                                    C::kThreads, 1, bb, pr, pk, det, s);
+        }
+        case 128: {
+            using C = fa::BwdCfg<128, 2>;
+            return launch_bwd_varlen<128, 128, BF16>(fa::bwd_kernel<128, 2, BF16, true, true>, C::kSmemBytes,
+                                                     C::kThreads, 1, bb, pr, pk, det, s);
+        }
+        case 256: {
+            using C = fa::BwdSplitCfg<256, 64, 2, 1, 2, true>;
+            return launch_bwd_varlen<256, 64, BF16>(fa::bwd_split_kernel<256, 64, 2, 1, 2, true, BF16, true, true>,
+                                                    C::kSmemBytes, C::kThreads, 2, bb, pr, pk, det, s);
+        }
+        default: return FA_ERR_UNSUPPORTED;
+    }
+}
+
 int bwd_varlen_impl(const BwdBuffers &bb, size_t workspace_bytes, const Problem &pr, const Packed &pk,
-                    void *stream) {
+                    void *stream, bool deterministic) {
     if (!bb.q || !bb.k || !bb.v || !bb.o || !bb.dout || !bb.lse || !bb.dq || !bb.dk || !bb.dv)
         return FA_ERR_INVALID_ARG;
     int rc = check_problem(pr);
     if (rc != FA_OK) return rc;
     if ((rc = check_packed(pk, pr)) != FA_OK) return rc;
-    if (pr.d == 256) return FA_ERR_UNSUPPORTED;
     const void *ptrs[] = {bb.q, bb.k, bb.v, bb.o, bb.dout, bb.lse, bb.dq, bb.dk, bb.dv};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
-    if (pr.BH() * ((pr.Nk + 127LL) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grid
+    if (pr.BH() * 2LL * ((pr.Nk + 127LL) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;   // one-dimensional grids
+    if (pr.BH() * ((pr.Nq + 127LL) / 128) > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     if (pr.BH() * fa::bwd_npad(pr.Nq) * (pr.d / 8) > 0x7fffffffLL * 256LL) return FA_ERR_UNSUPPORTED;
-    const size_t need = bwd_varlen_workspace_bytes(pr.BH(), pr.H, pk.total_q, pr.Nq, pr.d);
+    const size_t need = bwd_varlen_workspace_bytes(pr.BH(), pr.H, pk.total_q, pr.Nq, pr.d, deterministic);
     if (!bb.workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
     if (!aligned16(bb.workspace)) return FA_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (pr.dtype == FA_BF16)
-        return pr.d == 64 ? launch_bwd_varlen<64, true>(bb, pr, pk, s) : launch_bwd_varlen<128, true>(bb, pr, pk, s);
-    return pr.d == 64 ? launch_bwd_varlen<64, false>(bb, pr, pk, s) : launch_bwd_varlen<128, false>(bb, pr, pk, s);
+    if (pr.dtype == FA_BF16) return dispatch_bwd_varlen<true>(bb, pr, pk, deterministic, s);
+    return dispatch_bwd_varlen<false>(bb, pr, pk, deterministic, s);
 }
 
 // ---------------------------------------------------------------- fa_bwd_noalloc
@@ -732,9 +771,15 @@ FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, f
 }
 
 FA_API size_t fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d) {
-    if (B < 1 || H < 1 || total_q < 1 || max_seqlen_q < 1 || max_seqlen_q > total_q || (d != 64 && d != 128))
+    if (B < 1 || H < 1 || total_q < 1 || max_seqlen_q < 1 || max_seqlen_q > total_q ||
+        (d != 64 && d != 128 && d != 256))
         return 0;
-    return bwd_varlen_workspace_bytes(static_cast<long long>(B) * H, H, total_q, max_seqlen_q, d);
+    return bwd_varlen_workspace_bytes(static_cast<long long>(B) * H, H, total_q, max_seqlen_q, d, false);
+}
+
+FA_API size_t fa_bwd_varlen_deterministic_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d) {
+    if (fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_q, d) == 0) return 0;
+    return bwd_varlen_workspace_bytes(static_cast<long long>(B) * H, H, total_q, max_seqlen_q, d, true);
 }
 
 FA_API int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
@@ -746,7 +791,21 @@ FA_API int fa_bwd_varlen(const void *q, const void *k, const void *v, const void
                      nullptr, dtype};
     const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
     const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
-    return bwd_varlen_impl(bb, workspace_bytes, pr, pk, stream);
+    return bwd_varlen_impl(bb, workspace_bytes, pr, pk, stream, false);
+}
+
+FA_API int fa_bwd_varlen_deterministic(const void *q, const void *k, const void *v, const void *o,
+                                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                                       void *workspace, size_t workspace_bytes, const int *cu_seqlens_q,
+                                       const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                                       int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal,
+                                       int window_left, int window_right, const float *alibi_slopes, int dtype,
+                                       void *stream) {
+    const Problem pr{B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, window_left, window_right, alibi_slopes,
+                     nullptr, dtype};
+    const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+    const BwdBuffers bb{q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    return bwd_varlen_impl(bb, workspace_bytes, pr, pk, stream, true);
 }
 
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

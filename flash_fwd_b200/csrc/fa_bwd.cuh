@@ -169,10 +169,12 @@ __global__ void __launch_bounds__(256)
             acc = fmaf(x.x, y.x, acc);
             acc = fmaf(x.y, y.y, acc);
         }
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        const long long arow = static_cast<long long>(h) * total_q + t;
-        dqacc[(arow * D + part * 8) / 4] = z;
-        dqacc[(arow * D + part * 8) / 4 + 1] = z;
+        if (dqacc) {   // null: the deterministic backward keeps no accumulator
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            const long long arow = static_cast<long long>(h) * total_q + t;
+            dqacc[(arow * D + part * 8) / 4] = z;
+            dqacc[(arow * D + part * 8) / 4 + 1] = z;
+        }
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);

@@ -117,7 +117,7 @@ struct KIter {
 };
 
 // p.nqt counts 128-row query tiles here; p.dq receives dQ (16-bit, [BH][Nq][D]).
-template <int D, bool BF16, bool GENERAL>
+template <int D, bool BF16, bool GENERAL, bool VARLEN = false>
 __global__ void __launch_bounds__(352, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -132,10 +132,42 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    static_assert(GENERAL || !VARLEN, "packed batches use the general band");
     // one-dimensional grid, (batch, head) minor; the last query tiles see the
-    // most keys (causal, bottom-right bands), so they start first
-    const int bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
-    const int i = p.nqt - 1 - static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+    // most keys (causal, bottom-right bands), so they start first.  Packed
+    // batches: sequence major, then query tiles from the last, heads minor;
+    // a CTA past its own sequence's query tiles leaves before any setup.
+    // lp is p with the sequence's lengths; TMA rows are offset by qrow0 /
+    // krow0 in plane (the head)
+    int bh, i;
+    BwdParams lp;
+    int qrow0 = 0, krow0 = 0, plane = 0;
+    if constexpr (VARLEN) {
+        const unsigned per = static_cast<unsigned>(p.nqt) * static_cast<unsigned>(p.H);
+        const int b = static_cast<int>(blockIdx.x / per);
+        const int r = static_cast<int>(blockIdx.x - b * per);
+        const int ii = r / p.H;
+        plane = r - ii * p.H;
+        bh = b * p.H + plane;
+        const SeqSpan sq = seq_span(p.cu_q, b, p.total_q, p.Nq);
+        const SeqSpan sk = seq_span(p.cu_k, b, p.total_k, p.Nk);
+        const int nqt = (sq.len + 127) / 128;
+        if (ii >= nqt) return;
+        i = nqt - 1 - ii;
+        lp = p;
+        lp.Nq = sq.len;
+        lp.Nk = sk.len;
+        lp.nqt = nqt;
+        lp.nkb = (sk.len + 127) / 128;
+        lp.off = sk.len - sq.len;
+        qrow0 = sq.start;
+        krow0 = sk.start;
+    } else {
+        bh = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.nbh));
+        i = p.nqt - 1 - static_cast<int>(blockIdx.x / static_cast<unsigned>(p.nbh));
+        plane = bh;
+    }
+    const BwdParams &ip = pick<VARLEN>(lp, p);
 
     auto bar = [&](int x) -> uint32_t { return sbase + C::kBarOff + 8u * x; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -183,14 +215,14 @@ __global__ void __launch_bounds__(352, 1)
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTile);
             for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(sbase + C::kQOff + c * C::kChunk, &tmq, bar(C::kBarQ), c * 64, i * 128, bh);
-                tma_load_3d(sbase + C::kdOOff + c * C::kChunk, &tmdo, bar(C::kBarQ), c * 64, i * 128, bh);
+                tma_load_3d(sbase + C::kQOff + c * C::kChunk, &tmq, bar(C::kBarQ), c * 64, qrow0 + i * 128, plane);
+                tma_load_3d(sbase + C::kdOOff + c * C::kChunk, &tmdo, bar(C::kBarQ), c * 64, qrow0 + i * 128, plane);
             }
         }
         __syncwarp();
         KIter<GENERAL> it;
         int j;
-        while (it.next(p, i, j)) {
+        while (it.next(ip, i, j)) {
             if constexpr (C::kWide) {
                 // two halves of K_j, each refilled once the dQ half that reads it is done
                 for (int h = 0; h < 2 && ok; ++h) {
@@ -200,7 +232,7 @@ __global__ void __launch_bounds__(352, 1)
                         mbar_arrive_expect_tx(bar(C::kBarKFull + h), 2 * C::kChunk);
                         for (int c = 2 * h; c < 2 * h + 2; ++c)
                             tma_load_3d(sbase + C::kKOff + c * C::kChunk, &tmk, bar(C::kBarKFull + h), c * 64,
-                                        j * 128, bh);
+                                        krow0 + j * 128, plane);
                     }
                     __syncwarp();
                 }
@@ -213,7 +245,7 @@ __global__ void __launch_bounds__(352, 1)
                     mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTile);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(sbase + C::kKOff + s * C::kTile + c * C::kChunk, &tmk, bar(C::kBarKFull + s),
-                                    c * 64, j * 128, bh);
+                                    c * 64, krow0 + j * 128, plane);
                 }
                 __syncwarp();
             }
@@ -232,7 +264,7 @@ __global__ void __launch_bounds__(352, 1)
         constexpr int kLoadsPerBlock = C::kWide ? D / 64 : 1;
         KIter<GENERAL> it;
         int j;
-        while (ok && it.next(p, i, j)) {
+        while (ok && it.next(ip, i, j)) {
             for (int u = 0; u < kLoadsPerBlock; ++u) {   // cnt counts V slots filled
                 const int s = cnt % NSV;
                 ok = wait_bar(bar(C::kBarVEmpty + s), ((cnt / NSV) & 1) ^ 1u, abort_flag);
@@ -240,11 +272,12 @@ __global__ void __launch_bounds__(352, 1)
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kVSlot);
                     if constexpr (C::kWide) {
-                        tma_load_3d(sbase + C::kVOff + s * C::kVSlot, &tmv, bar(C::kBarVFull + s), u * 64, j * 128, bh);
+                        tma_load_3d(sbase + C::kVOff + s * C::kVSlot, &tmv, bar(C::kBarVFull + s), u * 64,
+                                    krow0 + j * 128, plane);
                     } else {
                         for (int c = 0; c < D / 64; ++c)
                             tma_load_3d(sbase + C::kVOff + s * C::kVSlot + c * C::kChunk, &tmv, bar(C::kBarVFull + s),
-                                        c * 64, j * 128, bh);
+                                        c * 64, krow0 + j * 128, plane);
                     }
                 }
                 __syncwarp();
@@ -292,7 +325,7 @@ __global__ void __launch_bounds__(352, 1)
 
         KIter<GENERAL> it;
         int jx;
-        bool have = it.next(p, i, jx);
+        bool have = it.next(ip, i, jx);
         if constexpr (C::kWide) {
             int nv = 0;   // V chunks consumed
             auto full_s = [&](int c) -> bool {   // S(c) from the two K halves
@@ -324,7 +357,7 @@ __global__ void __launch_bounds__(352, 1)
                 ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && full_s(0) && full_dp();
             }
             while (ok && have) {
-                const bool have_n = it.next(p, i, jx);
+                const bool have_n = it.next(ip, i, jx);
                 ok = wait_bar(bar(C::kBarDsFull), cnt & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -344,7 +377,7 @@ __global__ void __launch_bounds__(352, 1)
         } else {
             bool have_n = false;
             if (have) {
-                have_n = it.next(p, i, jx);
+                have_n = it.next(ip, i, jx);
                 ok = wait_bar(bar(C::kBarQ), 0, abort_flag) && wait_bar(bar(C::kBarKFull), 0, abort_flag) &&
                      wait_bar(bar(C::kBarVFull), 0, abort_flag);
                 if (ok) {
@@ -368,7 +401,7 @@ __global__ void __launch_bounds__(352, 1)
             }
             while (ok && have) {
                 const int c = cnt;
-                const bool have_nn = have_n && it.next(p, i, jx);
+                const bool have_nn = have_n && it.next(ip, i, jx);
                 if (have_n) {
                     // dP(c + 1) once the softmax-grad warps have read dP(c)
                     const int sv = (c + 1) % NSV;
@@ -419,7 +452,7 @@ __global__ void __launch_bounds__(352, 1)
         if (GENERAL && p.alibi) sl = -p.alibi[bh % p.H] / p.scale;
         KIter<GENERAL> it;
         int j;
-        while (it.next(p, i, j)) {
+        while (it.next(ip, i, j)) {
             const int b = cnt % NSB;
             const uint32_t ph = (cnt / NSB) & 1;
             const uint32_t tS = tmem + lane_off + C::kColS + 128 * b + 64 * kh;
@@ -429,9 +462,9 @@ __global__ void __launch_bounds__(352, 1)
             // keys kb0 + kk this row sees: lo <= kk <= hi (key q + off - wl ..
             // q + off + wr, below Nk); causal squares have off = 0, wr = 0
             const int kb0 = j * 128 + 64 * kh;
-            const int rk = q + p.off - kb0;   // |values| < 2^30 (Nq, Nk <= 2^28)
+            const int rk = q + ip.off - kb0;   // |values| < 2^30 (Nq, Nk <= 2^28)
             const int lo = max(rk - p.wl, -1);
-            const int hi = min(min(rk + p.wr, p.Nk - 1 - kb0), 64);
+            const int hi = min(min(rk + p.wr, ip.Nk - 1 - kb0), 64);
             float pv[64];
             {
                 uint32_t sr[64];
@@ -492,6 +525,10 @@ __global__ void __launch_bounds__(352, 1)
         // a tile that sees no key block never waited for its Q/dO loads: they
         // must land before the staging area (the Q buffer) is written
         if (done && cnt == 0) drain_bar(bar(C::kBarQ), 0);
+        // packed batches: a tile that ends inside the next sequence's rows is
+        // written row by row with plain stores (a TMA store clips only at the
+        // end of the tensor)
+        const int qrows = VARLEN ? ip.Nq - i * 128 : 128;
         if (done) {
             // this thread: row `row`, d columns [kh D / 2, (kh + 1) D / 2)
 #pragma unroll 1
@@ -508,6 +545,17 @@ __global__ void __launch_bounds__(352, 1)
                 for (int k = 0; k < 16; ++k)
                     pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * p.scale, __uint_as_float(v[2 * k + 1]) * p.scale);
                 const int col = kh * (D / 2) + 32 * ch;
+                if (VARLEN && qrows < 128) {
+                    if (row < qrows) {
+                        uint4 *g = reinterpret_cast<uint4 *>(
+                            static_cast<uint8_t *>(p.dq) +
+                            (static_cast<size_t>(qrow0 + i * 128 + row) * p.H + plane) * (D * 2) + col * 2);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            g[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                    }
+                    continue;
+                }
                 uint8_t *srow = smem + C::kQOff + (col / 64) * C::kChunk + row * 128;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -519,9 +567,9 @@ __global__ void __launch_bounds__(352, 1)
         }
         fence_async_smem();
         named_sync(1, 256);   // the eight softmax-grad warps (every one gets here)
-        if (done && warp == 0 && lane == 0) {
+        if (done && qrows >= 128 && warp == 0 && lane == 0) {
             for (int c = 0; c < D / 64; ++c)   // rows >= Nq are clipped
-                tma_store_3d(&tmdq, smem_u32(smem + C::kQOff + c * C::kChunk), c * 64, i * 128, bh);
+                tma_store_3d(&tmdq, smem_u32(smem + C::kQOff + c * C::kChunk), c * 64, qrow0 + i * 128, plane);
             bulk_commit();
             bulk_wait_read();
         }

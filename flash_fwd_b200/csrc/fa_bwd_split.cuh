@@ -64,7 +64,7 @@ struct BwdSplitCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16, bool GENERAL>
+template <int D, int BM, int DSPLIT, int NS, int NPB, bool DQT, bool BF16, bool GENERAL, bool VARLEN = false>
 __global__ void __launch_bounds__(320, 1)
     bwd_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
@@ -78,10 +78,19 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    static_assert(GENERAL || !VARLEN, "packed batches use the general band");
     // one-dimensional grid: groups of kHeadGroup heads, (batch, head) minor
-    // within a group (see bwd_kernel)
+    // within a group (see bwd_kernel).  Packed batches: sequence major, then
+    // (key block, column half), heads minor; a CTA past its own sequence's
+    // keys leaves before any setup.
     int bh, jh;
-    {
+    if constexpr (VARLEN) {
+        const long long per = static_cast<long long>(p.H) * p.nkb * DSPLIT;
+        const int b = static_cast<int>(blockIdx.x / per);
+        const int r = static_cast<int>(blockIdx.x - b * per);
+        jh = r / p.H;
+        bh = b * p.H + (r - jh * p.H);
+    } else {
         const int hg = min(C::kHeadGroup, p.nbh);
         const long long per = static_cast<long long>(hg) * p.nkb * DSPLIT;
         const int g = static_cast<int>(blockIdx.x / per);
@@ -92,6 +101,26 @@ __global__ void __launch_bounds__(320, 1)
     }
     const int j = jh / DSPLIT;
     const int h = jh % DSPLIT;
+    // packed batches: lp is p with this sequence's lengths; TMA rows are
+    // offset by qrow0 / krow0 in plane (the head)
+    BwdParams lp;
+    int qrow0 = 0, krow0 = 0, plane = bh;
+    if constexpr (VARLEN) {
+        const int b = bh / p.H;
+        plane = bh - b * p.H;
+        const SeqSpan sq = seq_span(p.cu_q, b, p.total_q, p.Nq);
+        const SeqSpan sk = seq_span(p.cu_k, b, p.total_k, p.Nk);
+        if (j * 128 >= sk.len) return;
+        lp = p;
+        lp.Nq = sq.len;
+        lp.Nk = sk.len;
+        lp.nqt = (sq.len + BM - 1) / BM;
+        lp.nkb = (sk.len + 127) / 128;
+        lp.off = sk.len - sq.len;
+        qrow0 = sq.start;
+        krow0 = sk.start;
+    }
+    const BwdParams &ip = pick<VARLEN>(lp, p);
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBarOff + 8u * i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::kMiscOff);
@@ -135,14 +164,16 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVTile);
             for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(sbase + C::kKOff + c * C::kKVChunk, &tmk, bar(C::kBarKV), c * 64, j * 128, bh);
-                tma_load_3d(sbase + C::kVOff + c * C::kKVChunk, &tmv, bar(C::kBarKV), c * 64, j * 128, bh);
+                tma_load_3d(sbase + C::kKOff + c * C::kKVChunk, &tmk, bar(C::kBarKV), c * 64, krow0 + j * 128,
+                            plane);
+                tma_load_3d(sbase + C::kVOff + c * C::kKVChunk, &tmv, bar(C::kBarKV), c * 64, krow0 + j * 128,
+                            plane);
             }
         }
         __syncwarp();
         QIter<BM, GENERAL> it;
         int i;
-        while (it.next(p, j, i)) {
+        while (it.next(ip, j, i)) {
             const int s = cnt % NS;
             const uint32_t ph = (cnt / NS) & 1;
             ok = wait_bar(bar(C::kBarQEmpty + s), ph ^ 1u, abort_flag);
@@ -153,8 +184,10 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t qb = bar(C::kBarQFull + s);
                 mbar_arrive_expect_tx(qb, 2 * C::kQTile + 2 * C::kStatBytes);
                 for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, qb, c * 64, i * BM, bh);
-                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo, qb, c * 64, i * BM, bh);
+                    tma_load_3d(sbase + C::kQOff + s * C::kQTile + c * C::kQChunk, &tmq, qb, c * 64,
+                                qrow0 + i * BM, plane);
+                    tma_load_3d(sbase + C::kdOOff + s * C::kQTile + c * C::kQChunk, &tmdo, qb, c * 64,
+                                qrow0 + i * BM, plane);
                 }
                 const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
                 bulk_load(sbase + C::kStatOff + s * 2 * C::kStatBytes, p.lse2 + srow, C::kStatBytes, qb);
@@ -226,7 +259,7 @@ __global__ void __launch_bounds__(320, 1)
 
         QIter<BM, GENERAL> it;
         int i, in;
-        bool have = it.next(p, j, i);
+        bool have = it.next(ip, j, i);
         if (have) {
             ok = wait_bar(bar(C::kBarKV), 0, abort_flag) && wait_bar(bar(C::kBarQFull), 0, abort_flag);
             if (ok) {
@@ -256,7 +289,7 @@ __global__ void __launch_bounds__(320, 1)
         while (ok && have) {
             const int s = cnt % NS;
             const int pb = cnt % NPB;
-            const bool have_n = it.next(p, j, in);
+            const bool have_n = it.next(ip, j, in);
             // with two or more stages the next tile is already resident: overlap
             // its S^T, dP^T with this tile's softmax-grad work.  With one stage
             // the next tile can only land after this tile's products finish.
@@ -301,7 +334,7 @@ __global__ void __launch_bounds__(320, 1)
         const float c = p.scale_log2;
         QIter<BM, GENERAL> it;
         int i;
-        while (it.next(p, j, i)) {
+        while (it.next(ip, j, i)) {
             const int s = cnt % NS;
             const int pb = cnt % NPB;
             uint8_t *sdS = smem + C::kdSOff + pb * C::kPTile;
@@ -317,10 +350,10 @@ __global__ void __launch_bounds__(320, 1)
             int qk, lo, hi;
             bool masked;
             if constexpr (GENERAL) {
-                qk = key - p.off - i * BM;     // |values| < 2^30 (Nq, Nk <= 2^28)
+                qk = key - ip.off - i * BM;     // |values| < 2^30 (Nq, Nk <= 2^28)
                 lo = max(qk - p.wr, -1);
                 hi = min(qk + p.wl, BM);
-                if (key >= p.Nk) lo = BM;
+                if (key >= ip.Nk) lo = BM;
                 masked = __any_sync(0xffffffffu, lo > 0 || hi < BM - 1);
             } else {
                 // square: queries before the key are hidden on the diagonal tiles
@@ -399,7 +432,7 @@ __global__ void __launch_bounds__(320, 1)
         const int t = (warp & 3) * 32 + lane;   // TMEM lane: a d index (transposed form) or a query row
         QIter<BM, GENERAL> it;
         int i;
-        while (it.next(p, j, i)) {
+        while (it.next(ip, j, i)) {
             if (p.dqacc == nullptr) {   // no dQ: only count the tiles (the dK epilogue needs cnt)
                 ++cnt;
                 continue;
@@ -412,17 +445,19 @@ __global__ void __launch_bounds__(320, 1)
             else tmem_ld128_wait(tmem + lane_off + C::kColDQ, v);
             tc_fence_before();
             mbar_arrive(bar(C::kBarDqEmpty));
-            float *accb = p.dqacc + static_cast<size_t>(bh) * p.Nq * D;
+            // accumulator rows of this (b, h): [BH][Nq][D], packed batches [H][total_q][D]
+            float *accb = p.dqacc + (VARLEN ? static_cast<size_t>(plane) * p.total_q + qrow0
+                                            : static_cast<size_t>(bh) * p.Nq) * D;
             if constexpr (DQT) {
                 const int dcol = h * DH + t;
 #pragma unroll
                 for (int k = 0; k < BM; ++k) {
                     const int q = i * BM + k;
-                    if (q < p.Nq) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
+                    if (q < ip.Nq) atomicAdd(accb + static_cast<size_t>(q) * D + dcol, __uint_as_float(v[k]));
                 }
             } else {
                 const int q = i * BM + t;
-                if (q < p.Nq) {
+                if (q < ip.Nq) {
                     float4 *dst = reinterpret_cast<float4 *>(accb + static_cast<size_t>(q) * D + h * DH);
 #pragma unroll
                     for (int k = 0; k < DH / 4; ++k)
@@ -451,6 +486,10 @@ __global__ void __launch_bounds__(320, 1)
         // a key block that no query tile sees never waited for its K/V loads:
         // they must land before the staging areas are written
         if (done && cnt == 0) drain_bar(bar(C::kBarKV), 0);
+        // packed batches: a key block that ends inside the next sequence's
+        // rows is written row by row with plain stores (a TMA store clips only
+        // at the end of the tensor)
+        const int krows = VARLEN ? ip.Nk - j * 128 : 128;
         if (done) {
 #pragma unroll 1
             for (int ch = 0; ch < DH / 32; ++ch) {
@@ -465,6 +504,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
                     pk[k] = pack2<BF16>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+                if (VARLEN && krows < 128) {
+                    if (r < krows) {
+                        uint4 *g = reinterpret_cast<uint4 *>(
+                            static_cast<uint8_t *>(is_dv ? p.dv : p.dk) +
+                            (static_cast<size_t>(krow0 + j * 128 + r) * p.H + plane) * (D * 2) + (h * DH + ch * 32) * 2);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            g[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                    }
+                    continue;
+                }
                 uint8_t *srow = stage + (ch >> 1) * C::kKVChunk + r * 128;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -476,9 +526,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         fence_async_smem();
         named_sync(is_dv ? 1 : 2, 128);   // the four warps of this output (every one gets here)
-        if (done && (warp & 3) == 0 && lane == 0) {
+        if (done && krows >= 128 && (warp & 3) == 0 && lane == 0) {
             for (int c = 0; c < DH / 64; ++c)   // keys >= Nk are clipped
-                tma_store_3d(is_dv ? &tmdv : &tmdk, smem_u32(stage + c * C::kKVChunk), h * DH + c * 64, j * 128, bh);
+                tma_store_3d(is_dv ? &tmdv : &tmdk, smem_u32(stage + c * C::kKVChunk), h * DH + c * 64,
+                             krow0 + j * 128, plane);
             bulk_commit();
             bulk_wait_read();
         }

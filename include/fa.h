@@ -188,20 +188,37 @@ FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, f
 /*
  * Workspace of fa_bwd_varlen: the two fp32 statistics [B][H][Npad] (Npad =
  * max_seqlen_q rounded up to FA_BLOCK) and the fp32 dQ accumulator
- * [H][total_q][d].  0 for invalid sizes (d = 256 included).
+ * [H][total_q][d].  0 for invalid sizes.
  */
 FA_API size_t fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d);
 
 /*
  * Backward of fa_fwd_varlen with the same arguments: dq [total_q][H][d],
- * dk, dv [total_k][H][d].  d = 64 or 128 (256: FA_ERR_UNSUPPORTED); dq is
- * accumulated with fp32 atomics as in fa_bwd.
+ * dk, dv [total_k][H][d], d = 64, 128 or 256.  dq is accumulated with fp32
+ * atomics as in fa_bwd.
  */
 FA_API int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const void *dout,
                          const float *lse, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
                          const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
                          int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal, int window_left,
                          int window_right, const float *alibi_slopes, int dtype, void *stream);
+
+/* Workspace of fa_bwd_varlen_deterministic: the two statistics only. */
+FA_API size_t fa_bwd_varlen_deterministic_workspace_bytes(int B, int H, int total_q, int max_seqlen_q, int d);
+
+/*
+ * fa_bwd_varlen with bitwise reproducible dq, dk, dv: as fa_bwd_deterministic,
+ * dQ is summed over each query tile's key blocks in a fixed order by a second
+ * pass instead of with atomics.  Same arguments as fa_bwd_varlen; the
+ * workspace is fa_bwd_varlen_deterministic_workspace_bytes().
+ */
+FA_API int fa_bwd_varlen_deterministic(const void *q, const void *k, const void *v, const void *o,
+                                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                                       void *workspace, size_t workspace_bytes, const int *cu_seqlens_q,
+                                       const int *cu_seqlens_k, int B, int H, int total_q, int total_k,
+                                       int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal,
+                                       int window_left, int window_right, const float *alibi_slopes, int dtype,
+                                       void *stream);
 
 /*
  * Bytes of device workspace fa_bwd_deterministic needs: the two fp32 per-row

@@ -2,9 +2,10 @@
 fa_bwd_varlen) with the fp64 oracle (oracle.fwd_varlen / bwd_varlen): B
 sequences of different lengths, including empty ones, single rows, exact
 tile multiples and ragged tails, concatenated along the token axis, in every
-mask mode, both 16-bit types and every head dim the entry points take.  Every
-element of O, LSE, dQ, dK, dV is compared; a sequence's partial last tile
-must not touch the rows of the sequence after it.
+mask mode, both 16-bit types and every head dim, for the default and the
+deterministic backward.  Every element of O, LSE, dQ, dK, dV is compared; a
+sequence's partial last tile must not touch the rows of the sequence after
+it.
 """
 import numpy as np
 import pytest
@@ -125,16 +126,54 @@ def test_varlen_equal_lengths_match_batched_entry_points():
     assert torch.equal(got[1].reshape(H, B, N).transpose(0, 1).contiguous(), lse.cpu())
 
 
-def test_varlen_bwd_d256_unsupported():
+@pytest.mark.parametrize("mode", ["dense", "causal", "window", "alibi"])
+@pytest.mark.parametrize("cross", [False, True])
+def test_varlen_fwd_bwd_d256(mode, cross):
+    H, d = 2, 256
+    lk = CROSS if cross else SELF
+    cu_q, cu_k, q, k, v, do = inputs.make_varlen(SELF, lk, H, d, "bf16", seed=21 + 3 * cross + len(mode))
+    m = MODES[mode]
+    slopes = inputs.alibi_slopes(H) if m.get("alibi") else None
+    scale = inputs.default_scale(d)
+    got = _gpu(cu_q, cu_k, q, k, v, do, m["causal"], scale, m.get("window"), slopes)
+    ref = oracle.bwd_varlen(q.double().numpy(), k.double().numpy(), v.double().numpy(), do.double().numpy(),
+                            cu_q.numpy(), cu_k.numpy(), scale, oracle.CAUSAL if m["causal"] else 0,
+                            window=m.get("window"), slopes=None if slopes is None else slopes.double().numpy())
+    _check(got, list(ref), "bf16")
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("mode", ["dense", "causal", "causal_window"])
+@pytest.mark.parametrize("cross", [False, True])
+def test_varlen_deterministic(d, mode, cross):
+    """fa_bwd_varlen_deterministic: the oracle's gradients, identical bytes on
+    a repeated call, and the same dK, dV bytes as the default backward."""
     import flash_fwd_b200 as fa
-    cu_q, cu_k, q, k, v, do = inputs.make_varlen([5, 9], [5, 9], 2, 256, "bf16")
+    H = 2
+    lk = CROSS if cross else SELF
+    cu_q, cu_k, q, k, v, do = inputs.make_varlen(SELF, lk, H, d, "bf16", seed=31 + d + len(mode) + 5 * cross)
+    m = MODES[mode]
+    scale = inputs.default_scale(d)
     dev = torch.device("cuda:0")
-    args = [t.to(dev) for t in (q, k, v)]
-    o, lse = fa.attention_fwd_varlen(*args, cu_q.to(dev), cu_k.to(dev), 9, 9)
-    with pytest.raises(fa.FaError) as e:
-        fa.attention_bwd_varlen(*args, o, do.to(dev), lse, cu_q.to(dev), cu_k.to(dev), 9, 9)
-    assert e.value.status == 2
+    cq, ck, qd, kd, vd, dod = (t.to(dev) for t in (cu_q, cu_k, q, k, v, do))
+    mq = int((cu_q[1:] - cu_q[:-1]).max())
+    mk = int((cu_k[1:] - cu_k[:-1]).max())
+    o, lse = fa.attention_fwd_varlen(qd, kd, vd, cq, ck, mq, mk, causal=m["causal"], scale=scale,
+                                     window=m.get("window"))
+    args = (qd, kd, vd, o, dod, lse, cq, ck, mq, mk)
+    kw = dict(causal=m["causal"], scale=scale, window=m.get("window"))
+    g1 = fa.attention_bwd_varlen(*args, deterministic=True, **kw)
+    g2 = fa.attention_bwd_varlen(*args, deterministic=True, **kw)
+    g0 = fa.attention_bwd_varlen(*args, **kw)
+    torch.cuda.synchronize()
     assert fa.fa_last_device_status() == 0
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    assert torch.equal(g1[1], g0[1]) and torch.equal(g1[2], g0[2])
+    ref = oracle.bwd_varlen(q.double().numpy(), k.double().numpy(), v.double().numpy(), do.double().numpy(),
+                            cu_q.numpy(), cu_k.numpy(), scale, oracle.CAUSAL if m["causal"] else 0,
+                            window=m.get("window"))
+    _check([o.cpu(), lse.cpu()] + [t.cpu() for t in g1], list(ref), "bf16")
 
 
 def test_varlen_bad_lengths_are_clamped_and_reported():
