@@ -19,6 +19,7 @@ __all__ = [
     "fa_bwd_deterministic_workspace_bytes", "fa_fp8_quantize_qkv", "fa_fwd_fp8", "attention_fwd_fp8",
     "fa_bwd_noalloc", "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_bytes", "attention_fwd_varlen",
     "attention_bwd_varlen", "fa_bwd_varlen_deterministic", "fa_bwd_varlen_deterministic_workspace_bytes",
+    "fa_selftest_wait_timeout",
 ]
 
 FA_BLOCK = 128
@@ -77,12 +78,14 @@ def load_library():
     lib.fa_last_device_status.argtypes = []
     lib.fa_version.argtypes = []
     lib.fa_last_timeout_site.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    lib.fa_selftest_wait_timeout.argtypes = [i, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
     lib.fa_profile_enable.argtypes = [i]
     lib.fa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
     for fn in (lib.fa_fwd, lib.fa_fwd_blocksparse, lib.fa_bwd, lib.fa_bwd_blocksparse, lib.fa_fwd_ex, lib.fa_bwd_ex,
                lib.fa_bwd_deterministic, lib.fa_fp8_quantize_qkv, lib.fa_fwd_fp8, lib.fa_bwd_noalloc,
                lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_bwd_varlen_deterministic,
-               lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read):
+               lib.fa_last_device_status, lib.fa_last_timeout_site, lib.fa_version, lib.fa_profile_enable, lib.fa_profile_read,
+               lib.fa_selftest_wait_timeout):
         fn.restype = ctypes.c_int
     _LIB = lib
     return lib
@@ -107,6 +110,20 @@ def fa_last_timeout_site():
 
 def fa_version():
     return load_library().fa_version()
+
+
+def fa_selftest_wait_timeout(warps, stream=None):
+    """Runs the failure self-test of the library (one CTA whose `warps` warps
+    wait, bounded, for an mbarrier phase that nothing completes) and returns
+    (status, site): FA_ERR_TIMEOUT (6) and the (block x, block y, warp,
+    mbarrier shared address, parity) of the wait that gave up.  Synchronises
+    the stream; takes about 3 s.  `stream` is a torch.cuda.Stream (None:
+    the current stream).  Without a GPU the library answers FA_ERR_CUDA
+    (FA_ERR_INVALID_ARG for a bad `warps`, checked first)."""
+    site = (ctypes.c_int * 5)()
+    s = _stream(stream) if torch.cuda.is_available() else ctypes.c_void_p(None)
+    rc = load_library().fa_selftest_wait_timeout(int(warps), s, site)
+    return rc, tuple(site)
 
 
 PROFILE_KINDS = ("fwd", "bwd_pre", "bwd_main", "bwd_post", "bwd_dq", "fp8_quant", "fwd_fp8")

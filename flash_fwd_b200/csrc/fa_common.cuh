@@ -19,8 +19,9 @@
 
 namespace fa {
 
-// Device error word (one per device that loads the library; every kernel of
-// the library is compiled into the one translation unit fa_api.cu).
+// Device error word (one per device that loads the library; every attention
+// kernel is compiled into the one translation unit fa_api.cu, and the
+// failure self-test of fa_selftest.cu has its own copy).
 static __device__ int g_dev_status = 0;
 // Where the first wait that gave up was: block x, block y, warp, shared
 // address of its mbarrier, parity waited for.  Written only by the thread

@@ -339,6 +339,27 @@ FA_API int fa_last_device_status(void);
 FA_API int fa_last_timeout_site(int *site);
 
 /*
+ * Failure-detection self-test.  Launches one CTA of `warps` warps (1 .. 32)
+ * on `stream` in which every warp waits, with the library's bounded wait,
+ * for an mbarrier phase that nothing completes; warp w starts its wait
+ * w x 100 ms after the CTA starts.  The first warp to reach the bound (3 s)
+ * raises the CTA's abort flag, which the other warps see at once although
+ * their own bounds have not run out, and records FA_ERR_TIMEOUT and where it
+ * waited; the kernel then returns (after about 3 s, not 3 s + 100 ms x
+ * (warps - 1)),
+ * with nothing in flight and the context usable.  The call synchronises the
+ * stream and returns the recorded status: FA_ERR_TIMEOUT when the wait gave
+ * up as designed (FA_OK would mean the wait completed: a defect).
+ * site[0..4] (a HOST array of 5 ints) receives block x, block y, warp,
+ * shared-memory address of the mbarrier and the parity waited for.  Uses its
+ * own copies of the device words: fa_last_device_status() and
+ * fa_last_timeout_site() are not touched.  FA_ERR_INVALID_ARG for warps
+ * outside 1 .. 32 or a null site, before anything is launched; FA_ERR_CUDA
+ * on a CUDA error.  Takes about 3 s.
+ */
+FA_API int fa_selftest_wait_timeout(int warps, void *stream, int *site);
+
+/*
  * Per-kernel timing, for benchmarks.  While enabled (on != 0), every call
  * records a pair of CUDA events on the caller's stream around each kernel it
  * launches.  fa_profile_read() waits for those events, writes the summed
