@@ -653,7 +653,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                     for (int k = 0; k < 128; ++k)
                         if (k < lo || k > hi) sv[k] = -INFINITY;
                 }
-                // row max: four independent chains of three-input max
+                // row max: four independent chains, two scores per step (fmax3)
                 float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
 #pragma unroll
                 for (int k = 4; k < 128; k += 8) {
@@ -681,11 +681,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, NSK, NSV>::kThreads, 1)
                 }
                 // P = 2^(s c - m).  kPolyPairs of every 8 pairs may go to the FMA
                 // pipe (polynomial) instead of the special-function unit.  Measured
-                // on B200: at d = 128 and 256 moving any pairs made the softmax
-                // slower (issue-bound); at d = 64 two of eight were 4.7 % faster
-                // but failed the parity of a causal cross-attention case (Nq = 300,
-                // Nk = 100) not yet explained, so every pair uses the special-
-                // function unit.
+                // on B200 with the persistent kernel: slower at every share tried
+                // (d = 128: one of eight pairs -4 %, two -7 %; d = 64: two of
+                // eight -2 %), so every pair uses the special-function unit.  (An
+                // earlier parity failure of the polynomial build was the
+                // three-input max of the row-max tree, now two-input, and rows
+                // with no visible key are recognised by their band limits.)
                 constexpr int kPolyPairs = 0;
                 float2 acc[4], acc_r[4];
 #pragma unroll
