@@ -183,3 +183,26 @@ def test_traffic_is_reported_only_for_unchanged_kernel_sources(tmp_path, monkeyp
     assert bench.traffic_for("bwd_main", "dsweep128") is None    # sources changed since the capture
     assert bench.traffic_for("fwd", "det128") is None            # never captured
     assert bench.traffic_for("fwd_fp8", "fp8_128") is None
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    src = ('// header comment\n#include "x.cuh"\n/* block\n comment */ int f(int a) {  \n'
+           '    const char *s = "// not a comment";   // trailing\n    char c = \'/\';\n\n    return a + 1;\n}\n')
+    assert bench.strip_comments(src) == ('#include "x.cuh"\n  int f(int a) {\n'
+                                         '    const char *s = "// not a comment";\n    char c = \'/\';\n    return a + 1;\n}')
+    csrc = tmp_path / "flash_fwd_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "fa_api.cu").write_text(src)
+    (csrc / "fa_common.cuh").write_text("int g;\n")
+    (csrc / "fa_selftest.cu").write_text("int h;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_sha()
+    (csrc / "fa_api.cu").write_text(src.replace("// trailing", "// another comment").replace("block", "other"))
+    assert bench.kernel_source_sha() == h0                # comments only
+    (csrc / "fa_selftest.cu").write_text("int h2;\n")
+    assert bench.kernel_source_sha() == h0                # the failure self-test is not a measured kernel
+    (csrc / "fa_api.cu").write_text(src.replace("a + 1", "a + 2"))
+    assert bench.kernel_source_sha() != h0                # code
+    (csrc / "fa_api.cu").write_text(src)
+    (csrc / "fa_common.cuh").write_text("int g2;\n")
+    assert bench.kernel_source_sha() != h0                # every header counts
