@@ -97,7 +97,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsweep128", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="wall-clock budget of the CPU oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -767,26 +767,57 @@ def run_ours(args, w, name):
         graph = {"error": str(e)[:200]}
 
     # ---------------- end to end through host buffers
+    # Every step copies its inputs from pinned host memory and its outputs back
+    # (PCIe: both directions at once).  Two device buffer sets alternate, so
+    # that the input copy of step i + 1 and the output copy of step i - 1 run
+    # beside the kernels of step i: inputs on one copy stream, outputs on
+    # another, kernels on the compute stream, ordered by events (a buffer set
+    # is refilled only after the kernels that read it, and its outputs are
+    # overwritten only after they were copied out).  The timed region runs
+    # from the first input copy to the last output copy.
     e2e = None
     if args.e2e_steps > 0:
-        pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "do", "cu_q", "cu_k") if host.get(n) is not None}
-        outs = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True)
-                for n in (["o", "lse", "dq", "dk", "dv"] if w["bwd"] else ["o", "lse"])}
+        in_names = [n for n in ("q", "k", "v", "do", "cu_q", "cu_k") if host.get(n) is not None]
+        out_names = ["o", "lse", "dq", "dk", "dv"] if w["bwd"] else ["o", "lse"]
+        pin = {n: host[n].pin_memory() for n in in_names}
+        outs = {n: torch.empty(t[n].shape, dtype=t[n].dtype, pin_memory=True) for n in out_names}
         h2d = sum(x.numel() * x.element_size() for x in pin.values())
         d2h = sum(x.numel() * x.element_size() for x in outs.values())
+        sets = [t, dict(t)]
+        for n in in_names + out_names:
+            sets[1][n] = torch.empty_like(t[n])
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        read = [None, None]     # per buffer set: its last kernels completed (inputs free)
+        drained = [None, None]  # per buffer set: its last outputs copied out
         fdist.barrier(device)
         torch.cuda.synchronize(device)
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(args.e2e_steps):
-            for n, x in pin.items():
-                t[n].copy_(x, non_blocking=True)
-            step(w, t, stream)
-            for n, x in outs.items():
-                x.copy_(t[n], non_blocking=True)
-        a1.record(stream)
+        a0.record(s_in)
+        for i in range(args.e2e_steps):
+            b = sets[i % 2]
+            if read[i % 2] is not None:
+                s_in.wait_event(read[i % 2])
+            with torch.cuda.stream(s_in):
+                for n in in_names:
+                    b[n].copy_(pin[n], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+            stream.wait_event(landed)
+            if drained[i % 2] is not None:
+                stream.wait_event(drained[i % 2])
+            step(w, b, stream)
+            read[i % 2] = torch.cuda.Event()
+            read[i % 2].record(stream)
+            s_out.wait_event(read[i % 2])
+            with torch.cuda.stream(s_out):
+                for n in out_names:
+                    outs[n].copy_(b[n], non_blocking=True)
+            drained[i % 2] = torch.cuda.Event()
+            drained[i % 2].record(s_out)
+        a1.record(s_out)
         torch.cuda.synchronize(device)
+        del sets
         e2e_ms = fdist.max_over_ranks(a0.elapsed_time(a1), device if args.gpus > 1 else None)
         e2e = {"value": fdist.aggregate_throughput([flops * args.e2e_steps] * world, e2e_ms) / 1e12,
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
